@@ -1,0 +1,299 @@
+// C ABI of the GVA decode library: argument validation, kernel selection, TMA
+// descriptor encoding and launches.  No allocation, no synchronisation.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace {
+
+thread_local char g_err[320] = "";
+
+gva_status_t fail(gva_status_t s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+gva_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(GVA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elt(int dtype) { return dtype == GVA_F32 ? 4 : 2; }
+
+bool dtype_ok(int d) { return d == GVA_F32 || d == GVA_BF16; }
+
+// SM count of the current device (cached per device).
+int num_sms() {
+  static int cache[64];
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+gva_status_t check_shape(const gva_shape_t* sh, bool gqa) {
+  if (!sh) return fail(GVA_ERR_INVALID_ARG, "shape is NULL");
+  if (sh->B < 0 || sh->B > gva::kMaxBatch)
+    return fail(GVA_ERR_INVALID_ARG, "B=%d outside [0, %d]", sh->B, gva::kMaxBatch);
+  if (sh->H < 1 || sh->G < 1 || sh->H % sh->G)
+    return fail(GVA_ERR_INVALID_ARG, "need H >= 1, G >= 1, H %% G == 0 (H=%d G=%d)", sh->H, sh->G);
+  if (sh->d_h < 1 || sh->d_h > 512) return fail(GVA_ERR_INVALID_ARG, "d_h=%d outside [1,512]", sh->d_h);
+  if (!gqa) {
+    if (sh->d_n < 0 || sh->d_n > 1024) return fail(GVA_ERR_INVALID_ARG, "d_n=%d outside [0,1024]", sh->d_n);
+    if (sh->d_r < 0 || sh->d_r > 256 || (sh->d_r & 1))
+      return fail(GVA_ERR_INVALID_ARG, "d_r=%d must be even and in [0,256]", sh->d_r);
+    if (!(sh->rope_base > 0.0) || !isfinite(sh->rope_base))
+      return fail(GVA_ERR_INVALID_ARG, "rope_base must be positive and finite");
+  }
+  if (!dtype_ok(sh->cache_dtype) || !dtype_ok(sh->q_dtype) || !dtype_ok(sh->out_dtype))
+    return fail(GVA_ERR_INVALID_ARG, "dtype codes must be GVA_F32 or GVA_BF16");
+  if (sh->softmax_scale < 0.f || !isfinite(sh->softmax_scale))
+    return fail(GVA_ERR_INVALID_ARG, "softmax_scale must be >= 0 and finite");
+  if (sh->ctas_per_sm < 0 || sh->ctas_per_sm > 32)
+    return fail(GVA_ERR_INVALID_ARG, "ctas_per_sm=%d outside [0,32]", sh->ctas_per_sm);
+  return GVA_OK;
+}
+
+float scale_of(const gva_shape_t& sh, bool gqa) {
+  if (sh.softmax_scale > 0.f) return sh.softmax_scale;
+  const int w = gqa ? sh.d_h : sh.d_n + sh.d_r;
+  return w > 0 ? (float)(1.0 / sqrt((double)w)) : 1.f;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 view [rows, cols] with row pitch `pitch_elems`, box [box_rows, box_cols].
+gva_status_t encode_2d(CUtensorMap* m, const void* base, long long rows, int cols, int pitch_elems,
+                       int box_rows, int box_cols, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(GVA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable from the driver");
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)pitch_elems * 2};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(GVA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) rows=%lld cols=%d box=%dx%d", (int)r,
+                rows, cols, box_rows, box_cols);
+  return GVA_OK;
+}
+
+struct Plan {
+  bool mma;
+  int grid;
+  gva::WsLayout ws;
+};
+
+gva_status_t plan_decode(const gva_shape_t& sh, bool gqa, long long max_total, Plan* p) {
+  const int sms = num_sms();
+  if (sms <= 0) return fail(GVA_ERR_CUDA, "no CUDA device");
+  p->mma = !(sh.flags & GVA_FLAG_FMA_PATH) && gva::mma_supported(sh, gqa);
+  p->grid = p->mma ? gva::mma_grid(sh, sms, max_total, gqa) : gva::simt_grid(sh, sms, max_total, gqa);
+  p->ws = gva::ws_layout(sh.B, sh.H, sh.d_h, p->grid);
+  return GVA_OK;
+}
+
+gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, const void* X,
+                           const void* Vv, const void* KR, const int32_t* seq_offset,
+                           const int32_t* seq_len, int64_t max_total_tokens, int64_t num_slots,
+                           void* out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  gva_status_t s = check_shape(shp, gqa);
+  if (s != GVA_OK) return s;
+  const gva_shape_t& sh = *shp;
+  if (sh.B == 0) return GVA_OK;
+  if (!q || !X || !Vv || !seq_offset || !seq_len || !out || !workspace)
+    return fail(GVA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!gqa && sh.d_r > 0 && !KR) return fail(GVA_ERR_INVALID_ARG, "kr_cache is NULL with d_r > 0");
+  if (!aligned16(q) || !aligned16(X) || !aligned16(Vv) || (KR && !aligned16(KR)) || !aligned16(out) ||
+      !aligned16(workspace) || !aligned16(seq_offset) || !aligned16(seq_len) || (lse && !aligned16(lse)))
+    return fail(GVA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (num_slots < 1 || num_slots >= (1ll << 31))
+    return fail(GVA_ERR_INVALID_ARG, "num_slots=%lld outside [1, 2^31)", (long long)num_slots);
+  if (max_total_tokens < 0 || max_total_tokens >= (1ll << 31))
+    return fail(GVA_ERR_INVALID_ARG, "max_total_tokens=%lld outside [0, 2^31)", (long long)max_total_tokens);
+  const int e = elt(sh.cache_dtype);
+  if ((sh.G * sh.d_h * e) % 16 || (!gqa && (sh.d_r * e) % 16))
+    return fail(GVA_ERR_INVALID_ARG, "cache rows must be multiples of 16 bytes (G*d_h*elt=%d, d_r*elt=%d)",
+                sh.G * sh.d_h * e, gqa ? 0 : sh.d_r * e);
+  Plan p;
+  if ((s = plan_decode(sh, gqa, max_total_tokens, &p)) != GVA_OK) return s;
+  if (ws_bytes < p.ws.total)
+    return fail(GVA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, p.ws.total);
+
+  gva::DecodeArgs a{};
+  a.B = sh.B;
+  a.H = sh.H;
+  a.G = sh.G;
+  a.d_h = sh.d_h;
+  a.d_r = gqa ? 0 : sh.d_r;
+  a.q_abs = gqa ? nullptr : static_cast<const float*>(q);
+  a.q_raw = gqa ? q : nullptr;
+  a.q_bf16 = sh.q_dtype == GVA_BF16;
+  a.q_scale = scale_of(sh, gqa) * gva::kLog2e;
+  a.X = X;
+  a.Vv = Vv;
+  a.KR = gqa ? nullptr : KR;
+  a.seq_offset = seq_offset;
+  a.seq_len = seq_len;
+  a.num_slots = num_slots;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.status = reinterpret_cast<int*>(ws);
+  a.meta = reinterpret_cast<int2*>(ws + p.ws.meta_off);
+  a.part_ml = reinterpret_cast<float2*>(ws + p.ws.ml_off);
+  a.part_o = reinterpret_cast<float*>(ws + p.ws.o_off);
+  a.grid = p.grid;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  cudaError_t err;
+  if (p.mma) {
+    a.tile = gva::mma_tile(sh, gqa);
+    const int tt = a.tile;
+    const int row = sh.G * sh.d_h;
+    CUtensorMap tx{}, tv{}, tk{};
+    if ((s = encode_2d(&tx, X, num_slots, row, row, tt, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != GVA_OK) return s;
+    tv = tx;
+    if (gqa && (s = encode_2d(&tv, Vv, num_slots, row, row, tt, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != GVA_OK)
+      return s;
+    tk = tx;
+    if (!gqa && sh.d_r > 0) {
+      const int drp = sh.d_r <= 16 ? 16 : 32;
+      if ((s = encode_2d(&tk, KR, num_slots, sh.d_r, sh.d_r, tt, drp,
+                         drp == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B)) != GVA_OK)
+        return s;
+    }
+    err = gva::launch_decode_mma(sh, gqa, a, tx, tv, tk, st);
+  } else {
+    a.tile = gva::simt_tile();
+    err = gva::launch_decode_simt(sh, gqa, a, st);
+    if (err == cudaErrorNotSupported)
+      return fail(GVA_ERR_UNSUPPORTED, "no decode kernel for H=%d G=%d d_h=%d d_r=%d", sh.H, sh.G,
+                  sh.d_h, sh.d_r);
+  }
+  if (err != cudaSuccess) return cuda_fail(err, "decode split kernel launch");
+  err = gva::launch_combine(sh, a, out, lse, st);
+  if (err != cudaSuccess) return cuda_fail(err, "combine kernel launch");
+  return GVA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gva_status_string(gva_status_t s) {
+  switch (s) {
+    case GVA_OK: return "ok";
+    case GVA_ERR_INVALID_ARG: return "invalid argument";
+    case GVA_ERR_UNSUPPORTED: return "unsupported shape";
+    case GVA_ERR_WORKSPACE: return "workspace too small";
+    case GVA_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+const char* gva_last_error(void) { return g_err; }
+
+gva_status_t gva_absorb_query(const gva_shape_t* shp, const void* q, const void* M,
+                              const int32_t* q_pos, float* q_abs, void* stream) {
+  gva_status_t s = check_shape(shp, false);
+  if (s != GVA_OK) return s;
+  const gva_shape_t& sh = *shp;
+  if (sh.B == 0) return GVA_OK;
+  if (!q || !q_abs || !q_pos || (sh.d_n > 0 && !M))
+    return fail(GVA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned16(q) || (M && !aligned16(M)) || !aligned16(q_pos) || !aligned16(q_abs))
+    return fail(GVA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const size_t smem = sizeof(float) * ((size_t)sh.d_h * (sh.d_n + 1) + sh.d_n + sh.d_r);
+  if (smem > 200 * 1024) return fail(GVA_ERR_UNSUPPORTED, "M_h too large for one CTA (%zu bytes)", smem);
+  const float c = scale_of(sh, false) * gva::kLog2e;
+  cudaError_t e = gva::launch_absorb(sh, q, M, q_pos, q_abs, c, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GVA_OK : cuda_fail(e, "absorb launch");
+}
+
+gva_status_t gva_append_cache(const gva_shape_t* shp, int32_t N, const void* v_new,
+                              const void* kpe_new, const int32_t* slot, const int32_t* pos,
+                              int64_t num_slots, void* V_cache, void* kr_cache, int32_t* err_flag,
+                              void* stream) {
+  gva_status_t s = check_shape(shp, false);
+  if (s != GVA_OK) return s;
+  const gva_shape_t& sh = *shp;
+  if (N < 0) return fail(GVA_ERR_INVALID_ARG, "N=%d < 0", N);
+  if (N == 0) return GVA_OK;
+  if (!v_new || !slot || !pos || !V_cache || (sh.d_r > 0 && (!kpe_new || !kr_cache)))
+    return fail(GVA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned16(v_new) || !aligned16(V_cache) || (kpe_new && !aligned16(kpe_new)) ||
+      (kr_cache && !aligned16(kr_cache)) || !aligned16(slot) || !aligned16(pos))
+    return fail(GVA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if ((sh.G * sh.d_h * elt(sh.cache_dtype)) % 16)
+    return fail(GVA_ERR_INVALID_ARG, "value rows must be multiples of 16 bytes");
+  if (num_slots < 1) return fail(GVA_ERR_INVALID_ARG, "num_slots=%lld < 1", (long long)num_slots);
+  cudaError_t e = gva::launch_append(sh, N, v_new, kpe_new, slot, pos, num_slots, V_cache, kr_cache,
+                                     err_flag, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GVA_OK : cuda_fail(e, "append launch");
+}
+
+size_t gva_decode_workspace_size(const gva_shape_t* shp, int64_t max_total_tokens) {
+  if (check_shape(shp, false) != GVA_OK && check_shape(shp, true) != GVA_OK) return 0;
+  if (max_total_tokens < 0) return 0;
+  size_t best = 0;
+  for (int gqa = 0; gqa < 2; ++gqa) {
+    if (check_shape(shp, gqa) != GVA_OK) continue;
+    Plan p;
+    if (plan_decode(*shp, gqa, max_total_tokens, &p) != GVA_OK) return 0;
+    if (p.ws.total > best) best = p.ws.total;
+  }
+  return best;
+}
+
+gva_status_t gva_decode_attention(const gva_shape_t* shape, const float* q_abs, const void* V_cache,
+                                  const void* kr_cache, const int32_t* seq_offset,
+                                  const int32_t* seq_len, int64_t max_total_tokens, int64_t num_slots,
+                                  void* out, float* lse, void* workspace, size_t ws_bytes,
+                                  void* stream) {
+  return decode_common(shape, false, q_abs, V_cache, V_cache, kr_cache, seq_offset, seq_len,
+                       max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream);
+}
+
+gva_status_t gqa_decode_attention(const gva_shape_t* shape, const void* q, const void* K_cache,
+                                  const void* V_cache, const int32_t* seq_offset,
+                                  const int32_t* seq_len, int64_t max_total_tokens, int64_t num_slots,
+                                  void* out, float* lse, void* workspace, size_t ws_bytes,
+                                  void* stream) {
+  return decode_common(shape, true, q, K_cache, V_cache, nullptr, seq_offset, seq_len,
+                       max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream);
+}
+
+}  // extern "C"

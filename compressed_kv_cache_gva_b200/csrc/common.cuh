@@ -1,0 +1,278 @@
+// Device helpers shared by the GVA decode kernels (sm_100a).
+//
+// Holds: the split-KV work list (token-balanced spans over a ragged batch), the
+// workspace layout, and thin inline-PTX wrappers for mbarrier, TMA bulk-tensor
+// loads, ldmatrix, movmatrix and the bf16 m16n8k16 tensor-core MMA.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gva.h"
+
+namespace gva {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kMaxBatch = 4096;          // sequences per call (prefix array lives in smem)
+constexpr uint32_t kWaitLimit = 1u << 22;  // iterations of a bounded mbarrier wait
+
+// ---------------------------------------------------------------------------
+// Workspace: [status word | meta[B] | partial (m,l)[P][H] | partial o[P][H][d_h]]
+// P = grid + B partial slots: the piece of sequence b handled by CTA i lands in
+// slot i + b (unique, see worklist below).
+// ---------------------------------------------------------------------------
+struct WsLayout {
+  size_t meta_off, ml_off, o_off, total;
+};
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline WsLayout ws_layout(int B, int H, int d_h, int grid) {
+  WsLayout w;
+  size_t parts = (size_t)grid + (size_t)B;
+  w.meta_off = 256;
+  w.ml_off = align_up(w.meta_off + sizeof(int2) * (size_t)B, 256);
+  w.o_off = align_up(w.ml_off + sizeof(float2) * parts * (size_t)H, 256);
+  w.total = align_up(w.o_off + sizeof(float) * parts * (size_t)H * (size_t)d_h, 256);
+  return w;
+}
+
+struct DecodeArgs {
+  int B, H, G, d_h, d_r;
+  const float* q_abs;        // GVA: [B,H,d_h+d_r] float32, pre-scaled to base-2 units
+  const void* q_raw;         // GQA: [B,H,d_h] q_dtype
+  int q_bf16;                // GQA: q stored as bf16 (else float32)
+  float q_scale;             // GQA: softmax_scale*log2(e); GVA: unused
+  const void* X;             // rows scored against the query: V (GVA) or K (GQA)
+  const void* Vv;            // value rows
+  const void* KR;            // GVA rotated positional key rows, or null
+  const int* seq_offset;
+  const int* seq_len;
+  long long num_slots;
+  int* status;
+  int2* meta;                // per sequence: (first partial slot, number of pieces)
+  float2* part_ml;           // [P][H] (running max, running sum), base-2
+  float* part_o;             // [P][H][d_h] un-normalised output
+  int grid;                  // CTAs of the split kernel
+  int tile;                  // span granularity in tokens
+};
+
+// ---------------------------------------------------------------------------
+// Split-KV work list.  Tokens of all sequences are concatenated in batch order;
+// CTA i owns the span [i*span, (i+1)*span) of that order with
+// span = ceil(total/grid) rounded up to `tile`.  The intersection of the span
+// with sequence b is one "piece"; it is written to partial slot i + b.  Two
+// non-empty pieces (b, i) and (b', i') with b + i = b' + i' cannot exist:
+// sequences are contiguous in the concatenated order, so b' > b forces i' >= i.
+// ---------------------------------------------------------------------------
+__device__ inline long long block_scan_lengths(const int* __restrict__ seq_len, int B,
+                                               int* prefix, long long* warp_tmp) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int per = (B + nt - 1) / nt;
+  const int beg = min(tid * per, B), end = min(beg + per, B);
+  long long sum = 0;
+  for (int b = beg; b < end; ++b) sum += max(__ldg(seq_len + b), 0);
+  const int lane = tid & 31, w = tid >> 5;
+  long long incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    long long v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_tmp[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    const int nw = (nt + 31) >> 5;
+    long long v = lane < nw ? warp_tmp[lane] : 0;
+    long long iv = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      long long u = __shfl_up_sync(0xffffffffu, iv, o);
+      if (lane >= o) iv += u;
+    }
+    if (lane < nw) warp_tmp[lane] = iv - v;
+    if (lane == nw - 1) warp_tmp[32] = iv;   // grand total
+  }
+  __syncthreads();
+  long long run = warp_tmp[w] + incl - sum;
+  const long long total = warp_tmp[32];
+  const bool fits = total < (1ll << 31);
+  for (int b = beg; b < end; ++b) {
+    prefix[b] = fits ? (int)run : 0;
+    run += max(__ldg(seq_len + b), 0);
+  }
+  if (tid == 0) prefix[B] = fits ? (int)total : 0;
+  __syncthreads();
+  return total;
+}
+
+struct Span {
+  int span;    // tokens per CTA
+  int total;   // tokens in the batch
+};
+
+__device__ inline Span make_span(int total, int grid, int tile) {
+  Span s;
+  s.total = total;
+  int per = (total + grid - 1) / grid;
+  s.span = max(tile, (per + tile - 1) / tile * tile);
+  return s;
+}
+
+// First sequence whose token range ends after `pos` (skips empty sequences).
+__device__ inline int seq_at(const int* prefix, int B, int pos) {
+  int lo = 0, hi = B;  // answer in [0, B]
+  while (lo < hi) {
+    int mid = (lo + hi) >> 1;
+    if (prefix[mid + 1] > pos) hi = mid; else lo = mid + 1;
+  }
+  return lo;
+}
+
+// CTA 0 records, for every sequence, where its pieces land and how many there are,
+// and flags sequences whose slots leave the cache.
+__device__ inline void write_meta(const DecodeArgs& a, const int* prefix, Span sp) {
+  for (int b = threadIdx.x; b < a.B; b += blockDim.x) {
+    int L = prefix[b + 1] - prefix[b];
+    int2 m = make_int2(0, 0);
+    if (L > 0) {
+      int first = prefix[b] / sp.span, last = (prefix[b + 1] - 1) / sp.span;
+      m = make_int2(first + b, last - first + 1);
+      long long off = __ldg(a.seq_offset + b);
+      if (off < 0 || off + L > a.num_slots) atomicOr(a.status, GVA_DEVERR_RANGE);
+    }
+    a.meta[b] = m;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Small numeric helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float ex2(float x) {  // 2^x on the SFU (PTX ex2.approx)
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float bf16_round(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
+
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+// ---------------------------------------------------------------------------
+// PTX wrappers (sm_90+/sm_100a)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: gives up after kWaitLimit polls and reports it in the status word.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* status) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  atomicOr(status, GVA_DEVERR_WAIT);
+  return false;
+}
+
+// 2-D tiled TMA load global -> shared, completion counted on an mbarrier.
+// No multicast: every CTA fetches its own tiles.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// D += A * B, m16n8k16, bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7},"
+      " {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Byte offset inside a TMA-swizzled tile: the 16-byte chunk index (bits 4..)
+// is XORed with bits 7.. of the offset; SW is the swizzle span in bytes.
+template <int SW>
+__device__ __forceinline__ uint32_t swz(uint32_t off) {
+  if constexpr (SW == 128) return off ^ ((off >> 3) & 0x70);
+  else if constexpr (SW == 64) return off ^ ((off >> 3) & 0x30);
+  else if constexpr (SW == 32) return off ^ ((off >> 3) & 0x10);
+  else return off;
+}
+
+}  // namespace gva

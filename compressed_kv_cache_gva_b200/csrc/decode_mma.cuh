@@ -1,0 +1,379 @@
+// Split-KV decode kernel on the tensor cores, TMA-staged (sm_100a).
+//
+// One CTA = NG consumer warps (warp g serves value group g and its HPG query
+// heads) + 1 producer warp that streams tiles of TT cache rows into a STAGES-deep
+// shared-memory ring with 2-D TMA loads (128-byte swizzle, no multicast) and
+// mbarrier completion.  Every tile is read from HBM once and serves all heads.
+//
+// Per tile and group (tokens on the MMA M axis, heads on N):
+//   scores  S[tok, n] = V_g[tok, :] . Qb[:, n]  (+ k_rope[tok, :] . Qr[:, n])
+//   softmax online in fp32, base 2 (the query is pre-scaled by scale*log2 e)
+//   output  O^T[d, n] += V_g^T[d, tok] . P[tok, n]
+// With HPG = 4 the 8 MMA columns hold [hi(q) of 4 heads | lo(q) of 4 heads],
+// q = hi + lo split into two bf16 numbers, so the fp32 query keeps ~16 bits of
+// significand at no extra MMA cost; P is split the same way for the second
+// product.  HPG = 8 uses two 8-column tiles (hi, lo).  The score fragment
+// (tokens on rows) is turned into the B operand of the second product
+// (tokens on K) with movmatrix.trans, so probabilities never touch shared memory.
+//
+// For GQA (same-shape comparison) the scores operand is the K tile, a separate V
+// tile is streamed next to it and there is no positional key.
+#pragma once
+
+#include "common.cuh"
+
+namespace gva {
+
+template <int D_H_, int NG_, int HPG_, int DRP_, bool GQA_>
+struct MmaCfg {
+  static constexpr int D_H = D_H_, NG = NG_, HPG = HPG_, DRP = GQA_ ? 0 : DRP_;
+  static constexpr bool GQA = GQA_;
+  static constexpr int ROW_BYTES = NG * D_H * 2 * (GQA ? 2 : 1);
+  static constexpr int TT_RAW = 16384 / ROW_BYTES;
+  static constexpr int TT = TT_RAW >= 64 ? 64 : (TT_RAW >= 32 ? 32 : 16);   // tokens per tile
+  static constexpr int CB = D_H / 64;                 // 64-column boxes per group
+  static constexpr int BOX = TT * 128;                // bytes of one [TT x 64] bf16 box
+  static constexpr int XB = NG * CB * BOX;            // scores operand (V or K)
+  static constexpr int VB = GQA ? XB : 0;             // separate value tile (GQA)
+  static constexpr int KRB = DRP ? TT * DRP * 2 : 0;  // positional key tile
+  static constexpr int STAGE = XB + VB + (KRB + 1023) / 1024 * 1024;
+  static constexpr int STAGES_RAW = (96 * 1024) / STAGE;
+  static constexpr int STAGES = STAGES_RAW < 2 ? 2 : (STAGES_RAW > 12 ? 12 : STAGES_RAW);
+  static constexpr int PIPE = STAGES * STAGE;
+  static constexpr uint32_t TX = XB + VB + KRB;       // bytes TMA delivers per stage
+  static constexpr int THREADS = (NG + 1) * 32;
+  static constexpr int NT = HPG == 8 ? 2 : 1;         // 8-column MMA tiles
+  static constexpr int KS = D_H / 16;                 // content k-steps (= d m-tiles)
+  static constexpr int RS = DRP / 16;                 // positional k-steps
+  static constexpr int MT = TT / 16;                  // 16-token m-tiles per tile
+  static constexpr int KR_SW = DRP * 2;               // swizzle span of the k_rope box
+  static_assert(HPG == 4 || HPG == 8, "heads per group");
+  static_assert(D_H % 64 == 0, "d_h");
+  static_assert(DRP == 0 || DRP == 16 || DRP == 32, "padded d_r");
+
+  static size_t smem_bytes(int B) {
+    return 1024 + PIPE + 16 * STAGES + sizeof(int) * (B + 1) + 16 + sizeof(long long) * 33;
+  }
+};
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS)
+    decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_x,
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_kr) {
+  extern __shared__ unsigned char smraw[];
+  uint8_t* pipe = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(pipe + C::PIPE);
+  uint64_t* empty = full + C::STAGES;
+  int* prefix = reinterpret_cast<int*>(empty + C::STAGES);
+  long long* wtmp = reinterpret_cast<long long*>(
+      (reinterpret_cast<uintptr_t>(prefix + a.B + 1) + 15) & ~uintptr_t(15));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(smem_u32(full + s), 1);
+      mbar_init(smem_u32(empty + s), C::NG);
+    }
+    fence_barrier_init();
+  }
+  if (warp == C::NG && lane == 0) {
+    prefetch_tmap(&tm_x);
+    if (C::GQA) prefetch_tmap(&tm_v);
+    if (C::DRP) prefetch_tmap(&tm_kr);
+  }
+  long long total64 = block_scan_lengths(a.seq_len, a.B, prefix, wtmp);   // syncs the block
+  int total = (int)total64;
+  if (total64 >= (1ll << 31)) {
+    if (threadIdx.x == 0) atomicOr(a.status, GVA_DEVERR_RANGE);
+    total = 0;
+  }
+  const Span sp = make_span(total, gridDim.x, C::TT);
+  if (blockIdx.x == 0) write_meta(a, prefix, sp);
+  const int s0 = blockIdx.x * sp.span;
+  if (s0 >= total) return;
+  const int s1 = min(s0 + sp.span, total);
+  const int b_first = seq_at(prefix, a.B, s0);
+
+  // ------------------------------------------------------------------ producer
+  if (warp == C::NG) {
+    if (lane != 0) return;
+    int k = 0;
+    bool ok = true;
+    for (int b = b_first; ok && b < a.B && prefix[b] < s1; ++b) {
+      const int j0 = max(s0, prefix[b]) - prefix[b], j1 = min(s1, prefix[b + 1]) - prefix[b];
+      const int row0 = __ldg(a.seq_offset + b);
+      for (int t0 = j0; t0 < j1; t0 += C::TT, ++k) {
+        const int s = k % C::STAGES;
+        if (k >= C::STAGES &&
+            !mbar_wait(smem_u32(empty + s), ((k / C::STAGES) - 1) & 1, a.status)) {
+          ok = false;
+          break;
+        }
+        const uint32_t fb = smem_u32(full + s);
+        mbar_arrive_expect_tx(fb, C::TX);
+        const uint32_t st = smem_u32(pipe + s * C::STAGE);
+        const int y = row0 + t0;
+#pragma unroll
+        for (int g = 0; g < C::NG; ++g)
+#pragma unroll
+          for (int c = 0; c < C::CB; ++c)
+            tma_load_2d(st + (g * C::CB + c) * C::BOX, &tm_x, g * C::D_H + c * 64, y, fb);
+        if constexpr (C::GQA) {
+#pragma unroll
+          for (int g = 0; g < C::NG; ++g)
+#pragma unroll
+            for (int c = 0; c < C::CB; ++c)
+              tma_load_2d(st + C::XB + (g * C::CB + c) * C::BOX, &tm_v, g * C::D_H + c * 64, y,
+                          fb);
+        }
+        if constexpr (C::DRP > 0) tma_load_2d(st + C::XB, &tm_kr, 0, y, fb);
+      }
+    }
+    // Drain: do not leave while a copy into this CTA's shared memory is in flight.
+    for (int kk = max(0, k - C::STAGES); kk < k; ++kk)
+      mbar_wait(smem_u32(full + kk % C::STAGES), (kk / C::STAGES) & 1, a.status);
+    return;
+  }
+
+  // ------------------------------------------------------------------ consumers
+  const int g = warp;
+  const int t = lane & 3, gq = lane >> 2;
+  const int mi = lane >> 3, r8 = lane & 7;
+  // ldmatrix row/chunk owned by this lane (see the fragment layouts of m16n8k16)
+  const int a_row = (mi & 1) * 8 + r8, a_kc = mi >> 1;     // scores A: rows=tokens
+  const int v_tok = (mi >> 1) * 8 + r8, v_dc = mi & 1;     // P.V A (trans): rows=tokens
+  const int H = a.H;
+  const int dq = C::D_H + a.d_r;
+  // columns owned after the hi/lo merge: heads h_lo, h_lo+1 of this group
+  const int hcol = (2 * t) & (C::HPG - 1);
+  const bool lo_half = (C::HPG == 4) && (t >= 2);
+
+  int k = 0;
+  for (int b = b_first; b < a.B && prefix[b] < s1; ++b) {
+    const int j0 = max(s0, prefix[b]) - prefix[b], j1 = min(s1, prefix[b + 1]) - prefix[b];
+    if (j1 <= j0) continue;
+
+    // ---- query fragments (B operand of the score MMA): column n = gq
+    uint32_t qb[C::NT][C::KS][2];
+    uint32_t qr[C::NT][C::RS > 0 ? C::RS : 1][2];
+#pragma unroll
+    for (int nt = 0; nt < C::NT; ++nt) {
+      const int hl = C::HPG == 8 ? gq : (gq & 3);
+      const bool lo = C::HPG == 8 ? (nt == 1) : (gq >= 4);
+      const int head = g * C::HPG + hl;
+      float v[C::KS][4];
+      float w[C::RS > 0 ? C::RS : 1][4];
+      if constexpr (!C::GQA) {
+        const float* qrow = a.q_abs + ((size_t)b * H + head) * dq;
+#pragma unroll
+        for (int ks = 0; ks < C::KS; ++ks) {
+          const int k0 = ks * 16 + 2 * t;
+          v[ks][0] = qrow[k0];
+          v[ks][1] = qrow[k0 + 1];
+          v[ks][2] = qrow[k0 + 8];
+          v[ks][3] = qrow[k0 + 9];
+        }
+#pragma unroll
+        for (int rs = 0; rs < C::RS; ++rs) {
+          const int k0 = rs * 16 + 2 * t;
+          const int kk[4] = {k0, k0 + 1, k0 + 8, k0 + 9};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) w[rs][e] = kk[e] < a.d_r ? qrow[C::D_H + kk[e]] : 0.f;
+        }
+      } else {
+        const size_t base = ((size_t)b * H + head) * C::D_H;
+#pragma unroll
+        for (int ks = 0; ks < C::KS; ++ks) {
+          const int k0 = ks * 16 + 2 * t;
+          const int kk[4] = {k0, k0 + 1, k0 + 8, k0 + 9};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float x = a.q_bf16
+                          ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.q_raw)[base + kk[e]])
+                          : reinterpret_cast<const float*>(a.q_raw)[base + kk[e]];
+            v[ks][e] = x * a.q_scale;
+          }
+        }
+      }
+      auto part = [&](float x) { float h = bf16_round(x); return lo ? x - h : h; };
+#pragma unroll
+      for (int ks = 0; ks < C::KS; ++ks) {
+        qb[nt][ks][0] = pack_bf16(part(v[ks][0]), part(v[ks][1]));
+        qb[nt][ks][1] = pack_bf16(part(v[ks][2]), part(v[ks][3]));
+      }
+#pragma unroll
+      for (int rs = 0; rs < C::RS; ++rs) {
+        qr[nt][rs][0] = pack_bf16(part(w[rs][0]), part(w[rs][1]));
+        qr[nt][rs][1] = pack_bf16(part(w[rs][2]), part(w[rs][3]));
+      }
+    }
+
+    float o[C::NT][C::KS][4];
+#pragma unroll
+    for (int nt = 0; nt < C::NT; ++nt)
+#pragma unroll
+      for (int md = 0; md < C::KS; ++md)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[nt][md][e] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+    for (int t0 = j0; t0 < j1; t0 += C::TT, ++k) {
+      const int s = k % C::STAGES;
+      if (!mbar_wait(smem_u32(full + s), (k / C::STAGES) & 1, a.status)) return;
+      const int nvalid = min(C::TT, j1 - t0);
+      uint8_t* st = pipe + s * C::STAGE;
+      uint8_t* xg = st + g * C::CB * C::BOX;
+      uint8_t* vg = C::GQA ? st + C::XB + g * C::CB * C::BOX : xg;
+      if (nvalid < C::TT) {
+        // rows past the sequence may hold anything (even NaN): zero them so
+        // that p = 0 really contributes nothing to P.V
+        const int nz = C::TT - nvalid;
+        for (int e = lane; e < nz * 8 * C::CB; e += 32) {
+          const int c = e / (nz * 8), rr = nvalid + (e >> 3) % nz, ch = e & 7;
+          *reinterpret_cast<uint4*>(vg + c * C::BOX + rr * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+      }
+      const uint32_t xg_u = smem_u32(xg), vg_u = smem_u32(vg), kr_u = smem_u32(st + C::XB);
+
+      // ---- scores
+      float sc[C::MT][4];
+#pragma unroll
+      for (int mt = 0; mt < C::MT; ++mt) {
+        float acc[C::NT][4];
+#pragma unroll
+        for (int nt = 0; nt < C::NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+        const int row = mt * 16 + a_row;
+#pragma unroll
+        for (int ks = 0; ks < C::KS; ++ks) {
+          uint32_t a0, a1, a2, a3;
+          const uint32_t addr = xg_u + (ks >> 2) * C::BOX + row * 128 +
+                                ((((ks & 3) * 2 + a_kc) ^ r8) << 4);
+          ldsm_x4(addr, a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < C::NT; ++nt) mma_bf16(acc[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
+        }
+#pragma unroll
+        for (int rs = 0; rs < C::RS; ++rs) {
+          uint32_t a0, a1, a2, a3;
+          const uint32_t addr = kr_u + swz<C::KR_SW>(row * C::DRP * 2 + (rs * 2 + a_kc) * 16);
+          ldsm_x4(addr, a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < C::NT; ++nt) mma_bf16(acc[nt], a0, a1, a2, a3, qr[nt][rs][0], qr[nt][rs][1]);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float x;
+          if constexpr (C::HPG == 8) x = acc[0][e] + acc[1][e];
+          else x = acc[0][e] + __shfl_xor_sync(0xffffffffu, acc[0][e], 2);
+          const int r = mt * 16 + gq + (e >= 2 ? 8 : 0);
+          sc[mt][e] = r < nvalid ? x : -INFINITY;
+        }
+      }
+
+      // ---- online softmax (fp32, base 2); this thread owns heads hcol, hcol+1
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int mt = 0; mt < C::MT; ++mt) {
+        mx0 = fmaxf(mx0, fmaxf(sc[mt][0], sc[mt][2]));
+        mx1 = fmaxf(mx1, fmaxf(sc[mt][1], sc[mt][3]));
+      }
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+      }
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
+      m0 = mn0;
+      m1 = mn1;
+      float rs0 = 0.f, rs1 = 0.f;
+      uint32_t bp[C::NT][C::MT][2];
+#pragma unroll
+      for (int mt = 0; mt < C::MT; ++mt) {
+        const float p0 = ex2(sc[mt][0] - m0), p1 = ex2(sc[mt][1] - m1);
+        const float p2 = ex2(sc[mt][2] - m0), p3 = ex2(sc[mt][3] - m1);
+        rs0 += p0 + p2;
+        rs1 += p1 + p3;
+        const float h0 = bf16_round(p0), h1 = bf16_round(p1), h2 = bf16_round(p2), h3 = bf16_round(p3);
+        if constexpr (C::HPG == 8) {
+          bp[0][mt][0] = movm_t(pack_bf16(h0, h1));
+          bp[0][mt][1] = movm_t(pack_bf16(h2, h3));
+          bp[1][mt][0] = movm_t(pack_bf16(p0 - h0, p1 - h1));
+          bp[1][mt][1] = movm_t(pack_bf16(p2 - h2, p3 - h3));
+        } else {
+          bp[0][mt][0] = movm_t(lo_half ? pack_bf16(p0 - h0, p1 - h1) : pack_bf16(h0, h1));
+          bp[0][mt][1] = movm_t(lo_half ? pack_bf16(p2 - h2, p3 - h3) : pack_bf16(h2, h3));
+        }
+      }
+      l0 = l0 * al0 + rs0;
+      l1 = l1 * al1 + rs1;
+#pragma unroll
+      for (int nt = 0; nt < C::NT; ++nt)
+#pragma unroll
+        for (int md = 0; md < C::KS; ++md) {
+          o[nt][md][0] *= al0;
+          o[nt][md][1] *= al1;
+          o[nt][md][2] *= al0;
+          o[nt][md][3] *= al1;
+        }
+
+      // ---- O^T += V^T P
+#pragma unroll
+      for (int mt = 0; mt < C::MT; ++mt) {
+        const int tok = mt * 16 + v_tok;
+#pragma unroll
+        for (int md = 0; md < C::KS; ++md) {
+          uint32_t a0, a1, a2, a3;
+          const uint32_t addr = vg_u + (md >> 2) * C::BOX + tok * 128 +
+                                ((((md & 3) * 2 + v_dc) ^ r8) << 4);
+          ldsm_x4_t(addr, a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < C::NT; ++nt)
+            mma_bf16(o[nt][md], a0, a1, a2, a3, bp[nt][mt][0], bp[nt][mt][1]);
+        }
+      }
+      if (nvalid < C::TT) fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(empty + s));
+    }
+
+    // ---- piece epilogue: un-normalised partial (m, l, o) to slot blockIdx.x + b
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+    }
+#pragma unroll
+    for (int md = 0; md < C::KS; ++md)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if constexpr (C::HPG == 8) o[0][md][e] += o[1][md][e];
+        else o[0][md][e] += __shfl_xor_sync(0xffffffffu, o[0][md][e], 2);
+      }
+    if (C::HPG == 8 || t < 2) {
+      const size_t slot = (size_t)blockIdx.x + b;
+      const int h0 = g * C::HPG + hcol;
+      float* po0 = a.part_o + (slot * H + h0) * C::D_H;
+      float* po1 = po0 + C::D_H;
+#pragma unroll
+      for (int md = 0; md < C::KS; ++md) {
+        const int d = md * 16 + gq;
+        po0[d] = o[0][md][0];
+        po1[d] = o[0][md][1];
+        po0[d + 8] = o[0][md][2];
+        po1[d + 8] = o[0][md][3];
+      }
+      if (gq == 0) {
+        a.part_ml[slot * H + h0] = make_float2(m0, l0);
+        a.part_ml[slot * H + h0 + 1] = make_float2(m1, l1);
+      }
+    }
+  }
+}
+
+}  // namespace gva

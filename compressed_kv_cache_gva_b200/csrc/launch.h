@@ -1,0 +1,39 @@
+// Internal launchers (host side), one per kernel family.  Called by api.cu after
+// argument validation; each returns the launch's cudaError_t.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/gva.h"
+
+namespace gva {
+
+struct DecodeArgs;
+
+cudaError_t launch_absorb(const gva_shape_t& sh, const void* q, const void* M, const int* q_pos,
+                          float* q_abs, float c, cudaStream_t st);
+
+cudaError_t launch_append(const gva_shape_t& sh, int N, const void* v_new, const void* kpe_new,
+                          const int* slot, const int* pos, long long num_slots, void* V_cache,
+                          void* kr_cache, int* err_flag, cudaStream_t st);
+
+// CUDA-core split kernel (any dtype / shape within limits).  Returns
+// cudaErrorNotSupported for shapes it is not built for.
+int simt_grid(const gva_shape_t& sh, int num_sms, long long max_total_tokens, bool gqa);
+int simt_tile();
+cudaError_t launch_decode_simt(const gva_shape_t& sh, bool gqa, DecodeArgs& a, cudaStream_t st);
+
+// Tensor-core split kernel with TMA staging (bf16 caches).
+bool mma_supported(const gva_shape_t& sh, bool gqa);
+int mma_grid(const gva_shape_t& sh, int num_sms, long long max_total_tokens, bool gqa);
+int mma_tile(const gva_shape_t& sh, bool gqa);
+cudaError_t launch_decode_mma(const gva_shape_t& sh, bool gqa, DecodeArgs& a,
+                              const CUtensorMap& tm_x, const CUtensorMap& tm_v,
+                              const CUtensorMap& tm_kr, cudaStream_t st);
+
+// Log-sum-exp combine of the partials into the output.
+cudaError_t launch_combine(const gva_shape_t& sh, const DecodeArgs& a, void* out, float* lse,
+                           cudaStream_t st);
+
+}  // namespace gva

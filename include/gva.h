@@ -1,0 +1,183 @@
+/*
+ * gva.h — C ABI of the B200 (sm_100a) Grouped Value Attention decode library.
+ *
+ * Grouped Value Attention (GVA) caches only the grouped values V[T,G,d_h] and one
+ * head-shared rotated positional key k_rope[T,d_r] per token.  Each query head h
+ * owns a fixed map M_h (d_h x d_n) with content key K_h = V_g(h) M_h; at decode the
+ * map is folded into the query, q~_h = q_h^nope M_h^T, so the score against cached
+ * token j is  s_j = (q~_h . v_{j,g(h)} + RoPE(q_h^rope) . k_rope_j) * scale  and the
+ * output is o_h = sum_j softmax(s)_j v_{j,g(h)}.  Content keys are never built.
+ *   - onedev.kr review "GVA는 값만 캐시하고 키를 필요할 때 복원해 GQA 캐시를 절반으로
+ *     줄인다", section "How it works" (어떻게 동작하나): K_h = V_g(h) M_h and the exact
+ *     absorption identity q_h (v M_h)^T = (q_h M_h^T) v^T;
+ *   - same review, section "What differs" (무엇과 다른가): decoupled RoPE slice d_r,
+ *     k_rope = (x_j W_r) R_j^T cached separately and shared by all heads, cache
+ *     N_GVA = T*G*d_h + T*d_r against N_GQA = 2*T*G*d_h;
+ *   - bisque.today explainer "Grouped Value Attention matches GQA on a 47% smaller KV
+ *     cache", Equation 7 (both routes give the same score, exactly).
+ *
+ * Conventions shared by every entry point
+ *   - The caller owns every buffer.  Pointers named "device" must point to device
+ *     memory of the current CUDA device; the library never allocates, frees or
+ *     synchronises, and keeps no per-call state.
+ *   - All work is enqueued asynchronously on `stream` (a cudaStream_t passed as
+ *     void*, NULL = legacy default stream).  Outputs are valid once the stream has
+ *     reached that point.
+ *   - Host-side validation happens before anything is launched; a non-OK status
+ *     means nothing was enqueued.  gva_last_error() returns a one-line reason for
+ *     the last non-OK status of the calling thread.  GVA_ERR_CUDA reports a launch
+ *     failure (cudaGetLastError after the launch).
+ *   - Layouts are dense row-major.  g(h) = h / (H/G) (contiguous grouping).
+ *     The query vector of a head is [content slice (d_n) | positional slice (d_r)].
+ *   - RoPE on the positional slice pairs element i with i + d_r/2 and rotates the
+ *     pair by pos * rope_base^(-2i/d_r); the angle is evaluated in float64.
+ *   - Sequence b owns cache slots seq_offset[b] .. seq_offset[b]+seq_len[b]-1, and
+ *     the token in slot seq_offset[b]+j has position j.  Sequences may be ragged.
+ */
+#ifndef GVA_H_
+#define GVA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GVA_OK = 0,
+  GVA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, inconsistent shape     */
+  GVA_ERR_UNSUPPORTED = 2,   /* valid shape that no kernel here is built for    */
+  GVA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required      */
+  GVA_ERR_CUDA = 4           /* a CUDA runtime call or launch failed            */
+} gva_status_t;
+
+typedef enum { GVA_F32 = 0, GVA_BF16 = 1 } gva_dtype_t;
+
+/* Flags for gva_shape_t.flags. */
+#define GVA_FLAG_FMA_PATH 1u   /* decode on CUDA-core FMA instead of tensor cores  */
+
+typedef struct {
+  int32_t B;            /* sequences (one query token each)                       */
+  int32_t H;            /* query heads                                            */
+  int32_t G;            /* value groups; H % G == 0                               */
+  int32_t d_h;          /* value / head width                                     */
+  int32_t d_n;          /* content (unrotated) query slice width                  */
+  int32_t d_r;          /* positional slice width, even, may be 0                 */
+  int32_t cache_dtype;  /* gva_dtype_t of V, k_rope (and K for GQA)               */
+  int32_t q_dtype;      /* gva_dtype_t of q and M                                 */
+  int32_t out_dtype;    /* gva_dtype_t of the attention output                    */
+  uint32_t flags;       /* GVA_FLAG_*                                             */
+  double rope_base;     /* RoPE base, e.g. 10000 or 500000                        */
+  float softmax_scale;  /* 0 -> 1/sqrt(d_n + d_r) (GVA) or 1/sqrt(d_h) (GQA)      */
+  int32_t ctas_per_sm;  /* split-KV CTAs per SM; 0 -> library default             */
+} gva_shape_t;
+
+/* One-line description of a status code (static storage). */
+const char* gva_status_string(gva_status_t status);
+
+/* Reason for the calling thread's most recent non-OK status (thread-local). */
+const char* gva_last_error(void);
+
+/*
+ * gva_absorb_query — fold each head's key map into its query and rotate the
+ * positional slice (onedev.kr review, "How it works": q~_h = q_h M_h^T is computed
+ * once per query token and head; "What differs": the positional slice is rotated).
+ *
+ *   q      device [B, H, d_n + d_r]  q_dtype
+ *   M      device [H, d_h, d_n]      q_dtype   (row i of M_h maps value dim i)
+ *   q_pos  device [B] int32          position of each sequence's query token
+ *   q_abs  device [B, H, d_h + d_r]  float32, written:
+ *            q_abs[b,h,0:d_h]      = c * (q[b,h,0:d_n] @ M[h]^T)
+ *            q_abs[b,h,d_h:d_h+d_r]= c * RoPE(q[b,h,d_n:], q_pos[b])
+ *          with c = softmax_scale * log2(e)  (scores come out in base-2 units).
+ * Alignment: every pointer 16-byte aligned.  Errors: GVA_ERR_INVALID_ARG.
+ */
+gva_status_t gva_absorb_query(const gva_shape_t* shape, const void* q, const void* M,
+                              const int32_t* q_pos, float* q_abs, void* stream);
+
+/*
+ * gva_append_cache — persist N new tokens: the grouped value is copied bit-exactly,
+ * the raw positional key is rotated by its own position and rounded once (to
+ * nearest, ties to even) to the cache type (onedev.kr review, "What differs":
+ * k_rope = (x_j W_r) R_j^T, cached separately, d_r scalars per token).
+ *
+ *   v_new    device [N, G, d_h]  cache_dtype
+ *   kpe_new  device [N, d_r]     cache_dtype, unrotated
+ *   slot     device [N] int32    destination slot of each token
+ *   pos      device [N] int32    position of each token (used by RoPE)
+ *   V_cache  device [num_slots, G, d_h]  cache_dtype, updated in place
+ *   kr_cache device [num_slots, d_r]     cache_dtype, updated in place
+ *   err_flag device int32 or NULL: set to 1 if any slot lies outside
+ *            [0, num_slots); such tokens are skipped, the others are written.
+ * Two tokens with the same slot race (last writer undefined).
+ * Alignment: 16 bytes for all cache/value pointers.  N == 0 is a no-op.
+ */
+gva_status_t gva_append_cache(const gva_shape_t* shape, int32_t N, const void* v_new,
+                              const void* kpe_new, const int32_t* slot, const int32_t* pos,
+                              int64_t num_slots, void* V_cache, void* kr_cache,
+                              int32_t* err_flag, void* stream);
+
+/*
+ * gva_decode_workspace_size — bytes of scratch gva_decode_attention and
+ * gqa_decode_attention need for `shape` on the CURRENT device (it depends on the
+ * device's SM count) when the total cached tokens never exceed max_total_tokens.
+ * Returns 0 for an invalid shape.
+ *
+ * Workspace contract: the first 4 bytes are a device status word.  Zero it once
+ * (e.g. cudaMemsetAsync of the whole buffer) before first use; the library never
+ * clears it.  After a decode it holds 0, or a nonzero GVA_DEVERR_* bit mask if a
+ * kernel met an inconsistent input (a sequence reaching outside [0, num_slots))
+ * or gave up a bounded wait.  The rest of the buffer is overwritten every call.
+ */
+size_t gva_decode_workspace_size(const gva_shape_t* shape, int64_t max_total_tokens);
+
+#define GVA_DEVERR_RANGE 1   /* some sequence's slots leave [0, num_slots); those rows read as 0 */
+#define GVA_DEVERR_WAIT 2    /* a pipeline wait hit its iteration limit; outputs invalid */
+
+/*
+ * gva_decode_attention — one GVA decode step over a (possibly ragged) batch,
+ * absorbed route (onedev.kr review, "How it works": content attention reads only
+ * the value cache, no key tensor; "What differs": plus the shared positional key).
+ * Split-KV over all SMs with a log-sum-exp combine.
+ *
+ *   q_abs      device [B, H, d_h + d_r] float32 from gva_absorb_query
+ *   V_cache    device [num_slots, G, d_h] cache_dtype
+ *   kr_cache   device [num_slots, d_r]    cache_dtype, already rotated (ignored if d_r==0)
+ *   seq_offset device [B] int32, seq_len device [B] int32 (0 allowed)
+ *   max_total_tokens  upper bound of sum(seq_len) (host value, sizes the split)
+ *   out        device [B, H, d_h] out_dtype   o_h = sum_j p_j v_{j,g(h)}
+ *   lse        device [B, H] float32 or NULL: natural-log log-sum-exp of the scaled
+ *              scores (-inf for an empty sequence, whose output is 0)
+ *   workspace  device, ws_bytes >= gva_decode_workspace_size(shape, max_total_tokens)
+ * Alignment: 16 bytes for all pointers; V_cache rows (G*d_h*elt) and k_rope rows
+ * (d_r*elt) must be multiples of 16 bytes.  Concurrent calls on different streams
+ * must use different workspaces.
+ */
+gva_status_t gva_decode_attention(const gva_shape_t* shape, const float* q_abs,
+                                  const void* V_cache, const void* kr_cache,
+                                  const int32_t* seq_offset, const int32_t* seq_len,
+                                  int64_t max_total_tokens, int64_t num_slots, void* out,
+                                  float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * gqa_decode_attention — same-shape grouped-query attention decode, the matched
+ * baseline of every page (it caches a key AND a value per group and token,
+ * N_GQA = 2*T*G*d_h).  Same split and combine as gva_decode_attention.
+ *
+ *   q          device [B, H, d_h] q_dtype, already rotated
+ *   K_cache, V_cache  device [num_slots, G, d_h] cache_dtype (keys already rotated)
+ *   scale      shape->softmax_scale, 0 -> 1/sqrt(d_h); shape->d_n and d_r are ignored
+ * Other arguments, alignment and workspace as for gva_decode_attention.
+ */
+gva_status_t gqa_decode_attention(const gva_shape_t* shape, const void* q, const void* K_cache,
+                                  const void* V_cache, const int32_t* seq_offset,
+                                  const int32_t* seq_len, int64_t max_total_tokens,
+                                  int64_t num_slots, void* out, float* lse, void* workspace,
+                                  size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* GVA_H_ */

@@ -1,0 +1,121 @@
+"""The C ABI library: it builds, loads, exports every symbol the header
+declares, and validates arguments on the host (CPU only, no kernel runs)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from compressed_kv_cache_gva_b200 import _build, gva
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gva.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    _build.build()
+    return gva.lib()
+
+
+def declared_functions():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\**(\w+)\s*\(", txt, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("gva_absorb_query", "gva_append_cache", "gva_decode_attention",
+              "gqa_decode_attention", "gva_decode_workspace_size", "gva_status_string",
+              "gva_last_error"):
+        assert n in names, n
+
+
+def test_every_declared_symbol_is_exported(L):
+    for n in declared_functions():
+        assert hasattr(L, n), f"{n} declared in gva.h but not exported"
+    assert sorted(gva.EXPORTS) == declared_functions()
+
+
+def test_shape_struct_layout():
+    # gva_shape_t: 10 x 4-byte fields, a double at offset 40, float + int32 after it
+    assert ctypes.sizeof(gva.Shape) == 56
+    assert gva.Shape.rope_base.offset == 40
+    assert gva.Shape.softmax_scale.offset == 48
+
+
+def test_status_strings(L):
+    for code, text in [(0, b"ok"), (1, b"invalid argument"), (2, b"unsupported shape"),
+                       (3, b"workspace too small"), (4, b"CUDA error")]:
+        assert L.gva_status_string(code) == text
+
+
+def _shape(**kw):
+    base = dict(B=2, H=16, G=4, d_h=64, d_n=48, d_r=16)
+    base.update(kw)
+    return gva.make_shape(**base)
+
+
+FAKE = 1 << 20    # never dereferenced: validation rejects before any CUDA call
+
+
+@pytest.mark.parametrize("bad", [dict(H=15), dict(G=0), dict(d_r=15), dict(d_h=0), dict(B=-1),
+                                 dict(B=5000), dict(d_r=-2), dict(rope_base=0.0),
+                                 dict(softmax_scale=-1.0), dict(ctas_per_sm=99)])
+def test_invalid_shapes_are_rejected(L, bad):
+    sh = _shape(**bad)
+    st = L.gva_decode_attention(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, FAKE, 100, 100, FAKE, None,
+                                FAKE, 1 << 20, None)
+    assert st == 1
+    assert L.gva_last_error()
+    assert L.gva_decode_workspace_size(ctypes.byref(sh), 100) == 0 or bad.keys() <= {"d_r", "rope_base"}
+
+
+def test_null_and_misaligned_pointers(L):
+    sh = _shape()
+    st = L.gva_decode_attention(ctypes.byref(sh), None, FAKE, FAKE, FAKE, FAKE, 100, 100, FAKE, None,
+                                FAKE, 1 << 20, None)
+    assert st == 1 and b"NULL" in L.gva_last_error()
+    st = L.gva_decode_attention(ctypes.byref(sh), FAKE + 4, FAKE, FAKE, FAKE, FAKE, 100, 100, FAKE,
+                                None, FAKE, 1 << 20, None)
+    assert st == 1 and b"aligned" in L.gva_last_error()
+    st = L.gva_absorb_query(ctypes.byref(sh), FAKE, FAKE + 8, FAKE, FAKE, None)
+    assert st == 1
+    st = L.gva_append_cache(ctypes.byref(sh), 4, FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE, None, None)
+    assert st == 1 and b"num_slots" in L.gva_last_error()
+    st = L.gva_append_cache(ctypes.byref(sh), -1, FAKE, FAKE, FAKE, FAKE, 10, FAKE, FAKE, None, None)
+    assert st == 1
+
+
+def test_bad_sizes(L):
+    sh = _shape()
+    st = L.gva_decode_attention(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, FAKE, 100, 0, FAKE, None,
+                                FAKE, 1 << 20, None)
+    assert st == 1 and b"num_slots" in L.gva_last_error()
+    st = L.gva_decode_attention(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 31, 100, FAKE,
+                                None, FAKE, 1 << 20, None)
+    assert st == 1 and b"max_total_tokens" in L.gva_last_error()
+    sh = _shape(G=3, H=12, d_h=40, d_r=6)      # rows of 240 B ok, k_rope rows of 12 B are not
+    st = L.gva_decode_attention(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, FAKE, 100, 100, FAKE, None,
+                                FAKE, 1 << 20, None)
+    assert st == 1 and b"16 bytes" in L.gva_last_error()
+
+
+def test_empty_batch_and_empty_append_are_noops(L):
+    sh = _shape(B=0)
+    assert L.gva_decode_attention(ctypes.byref(sh), None, None, None, None, None, 0, 1, None, None,
+                                  None, 0, None) == 0
+    sh = _shape()
+    assert L.gva_append_cache(ctypes.byref(sh), 0, None, None, None, None, 1, None, None, None,
+                              None) == 0
+
+
+def test_no_device_is_a_cuda_error_not_a_crash(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    sh = _shape()
+    st = L.gva_decode_attention(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, FAKE, 100, 100, FAKE, None,
+                                FAKE, 1 << 20, None)
+    assert st == 4

@@ -1,0 +1,237 @@
+"""CUDA path against the float64 oracle, element by element, through the C ABI.
+
+Workloads are the five GVA decode shapes (reduced cache lengths here so the
+oracle runs in seconds while still spanning many tiles and ragged tails; the
+full sizes run in test_gpu_full_size.py on sampled outputs)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from compressed_kv_cache_gva_b200 import gva
+from compressed_kv_cache_gva_b200.synth import (WORKLOADS, as_f64, make_append_inputs,
+                                                make_decode_inputs, make_gqa_inputs)
+from gpu_helpers import (LOG2E, assert_close, dev, lse_close, oracle_gqa, oracle_gva, run_gqa,
+                         run_gva, shape_of)
+
+pytestmark = pytest.mark.gpu
+
+NAMES = list(WORKLOADS)
+
+
+def small(name, lengths=None):
+    """The workload with short caches: lengths that cross tile boundaries and
+    leave ragged tails (tiles are 16, 32 or 64 rows)."""
+    wl = WORKLOADS[name]
+    if lengths is None:
+        if wl.dtype == "f32":
+            lengths = [64]
+        else:
+            base = [1, 15, 16, 17, 31, 33, 63, 65, 100, 257, 640, 1031]
+            lengths = base[:max(2, min(len(base), wl.B + 4))]
+    return make_decode_inputs(wl, extra_slots=1, lengths=np.array(lengths))
+
+
+# ------------------------------------------------------------------ absorb
+
+@pytest.mark.parametrize("name", NAMES)
+def test_absorb_query(name):
+    di = small(name)
+    wl = di.wl
+    _, _, q_abs, _ = run_gva(di)
+    qt, qr = oracle.absorbed_query(as_f64(di.q), as_f64(di.M), di.q_pos.numpy(), wl.d_n, wl.d_r,
+                                   wl.rope_base)
+    c = LOG2E / math.sqrt(wl.d_n + wl.d_r)
+    got_t = q_abs[:, :, :wl.d_h] / c
+    got_r = q_abs[:, :, wl.d_h:] / c
+    for got, ref in ((got_t, qt), (got_r, qr)):
+        err = np.max(np.abs(got - ref)) / max(1.0, np.max(np.abs(ref)))
+        assert err < 2e-6, err
+
+
+# ------------------------------------------------------------------ append
+
+@pytest.mark.parametrize("name", NAMES)
+def test_append_cache(name):
+    wl = WORKLOADS[name]
+    di = make_decode_inputs(wl, extra_slots=2, lengths=np.array([5, 40, 3]))
+    S = di.num_slots
+    rng = np.random.default_rng(5)
+    slots = rng.choice(S, size=24, replace=False).astype(np.int32)
+    pos = rng.integers(0, 131072 * 2, size=24).astype(np.int32)
+    slots[3] = S          # out of range: skipped, flagged
+    slots[7] = -1
+    ap = make_append_inputs(wl, slots, pos)
+    V, KR = dev(di.V), dev(di.k_rope)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sh = shape_of(di)
+    gva.append_cache(sh, dev(ap.v_new), dev(ap.kpe_new), dev(ap.slot), dev(ap.pos), V, KR, err)
+    torch.cuda.synchronize()
+    V_ref, K_ref, e_ref = oracle.append_cache(as_f64(di.V), as_f64(di.k_rope), as_f64(ap.v_new),
+                                              as_f64(ap.kpe_new), slots, pos, wl.rope_base, wl.dtype)
+    assert int(err.item()) == e_ref == 1
+    # values: a bit-exact copy; untouched rows unchanged
+    assert np.array_equal(as_f64(V.cpu()), V_ref)
+    # rotated keys: both sides round the float64 rotation once to the cache type;
+    # the only admissible difference is a tie decided differently by the last
+    # float64 bit, which never happened on these draws
+    got = as_f64(KR.cpu())
+    same = got == K_ref
+    assert same.all(), f"{(~same).sum()} rotated-key elements differ"
+
+
+def test_append_then_decode_end_to_end():
+    """Raw keys through the GPU append, then GPU decode, against the oracle's
+    append followed by the oracle's decode."""
+    wl = WORKLOADS["350m_b8_t4096"]
+    lengths = np.array([70, 129, 1])
+    di = make_decode_inputs(wl, extra_slots=1, lengths=lengths)
+    V0, K0 = as_f64(di.V), as_f64(di.k_rope)
+    offs = di.seq_offset.numpy()
+    slots = (offs + lengths).astype(np.int32)
+    ap = make_append_inputs(wl, slots, lengths.astype(np.int32))
+    V, KR = dev(di.V), dev(di.k_rope)
+    sh = shape_of(di)
+    gva.append_cache(sh, dev(ap.v_new), dev(ap.kpe_new), dev(ap.slot), dev(ap.pos), V, KR)
+    torch.cuda.synchronize()
+    di.V, di.k_rope = V.cpu(), KR.cpu()
+    di.seq_len = torch.from_numpy((lengths + 1).astype(np.int32))
+    di.q_pos = di.seq_len.clone() - 1      # the new token queries at its own position
+    out, lse, _, st = run_gva(di)
+    V_ref, K_ref, _ = oracle.append_cache(V0, K0, as_f64(ap.v_new), as_f64(ap.kpe_new), slots, lengths,
+                                          wl.rope_base, wl.dtype)
+    ref, ref_lse = oracle.gva_decode(as_f64(di.q), as_f64(di.M), di.q_pos.numpy(), V_ref, K_ref,
+                                     offs, di.seq_len.numpy(), wl.d_n, wl.d_r, wl.rope_base)
+    assert st == 0
+    assert_close(out, ref, wl.dtype, "append+decode")
+    lse_close(lse, ref_lse)
+
+
+# ------------------------------------------------------------------ decode
+
+@pytest.mark.parametrize("flags", [0, gva.FLAG_FMA_PATH], ids=["tensor", "fma"])
+@pytest.mark.parametrize("name", NAMES)
+def test_decode_matches_oracle(name, flags):
+    di = small(name)
+    out, lse, _, st = run_gva(di, flags=flags)
+    ref, ref_lse = oracle_gva(di)
+    assert st == 0
+    assert_close(out, ref, di.wl.dtype, name)
+    lse_close(lse, ref_lse, name)
+
+
+def test_decode_fp32_ragged():
+    di = small("tiny_fp32_t64", lengths=[64, 1, 17, 100, 0, 33])
+    for flags in (0, gva.FLAG_FMA_PATH):
+        out, lse, _, st = run_gva(di, flags=flags)
+        ref, ref_lse = oracle_gva(di)
+        assert st == 0
+        assert_close(out, ref, "f32")
+        lse_close(lse, ref_lse)
+
+
+@pytest.mark.parametrize("cps", [1, 2, 3])
+def test_decode_split_counts_agree(cps):
+    """The split changes with CTAs per SM; the answer does not."""
+    di = small("350m_b8_t4096", lengths=[4096, 777, 2048])
+    out, lse, _, st = run_gva(di, ctas_per_sm=cps)
+    ref, ref_lse = oracle_gva(di)
+    assert st == 0
+    assert_close(out, ref, "bf16", f"cps={cps}")
+
+
+@pytest.mark.parametrize("lengths", [[0], [0, 0, 0], [1], [0, 5, 0, 1], [16, 0, 17], [33] * 9,
+                                     [1] * 300], ids=["empty", "all-empty", "one", "mixed-empty",
+                                                      "tile-edges", "many-small", "300x1"])
+def test_decode_edge_lengths(lengths):
+    di = small("350m_b8_t4096", lengths=lengths)
+    out, lse, _, st = run_gva(di)
+    ref, ref_lse = oracle_gva(di)
+    assert st == 0
+    L = np.array(lengths)
+    assert np.all(out[L == 0] == 0)
+    assert np.all(np.isneginf(lse[L == 0]))
+    assert_close(out, ref, "bf16")
+    lse_close(lse, ref_lse)
+
+
+def test_decode_length_one_returns_the_value_row():
+    di = small("350m_b8_t4096", lengths=[1, 1])
+    out, _, _, _ = run_gva(di)
+    V = as_f64(di.V)
+    for b in range(2):
+        for h in range(16):
+            np.testing.assert_allclose(out[b, h], V[di.seq_offset[b].item(), h // 4], rtol=0, atol=1e-6)
+
+
+def test_decode_large_batch_scan():
+    """4096 sequences exercise the in-kernel length scan over many threads."""
+    rng = np.random.default_rng(3)
+    lengths = rng.integers(0, 24, size=4096)
+    di = small("350m_b8_t4096", lengths=lengths)
+    pairs = [(b, h) for b in rng.choice(4096, 40, replace=False) for h in (0, 7, 15)]
+    out, lse, _, st = run_gva(di)
+    ref, ref_lse = oracle_gva(di, pairs=pairs)
+    assert st == 0
+    idx = tuple(np.array(pairs).T)
+    assert_close(out[idx], ref[idx], "bf16")
+
+
+def test_decode_bf16_output():
+    di = small("350m_b8_t4096")
+    out, _, _, _ = run_gva(di, out_dtype=torch.bfloat16)
+    ref, _ = oracle_gva(di)
+    assert_close(out, ref, "bf16")
+
+
+def test_decode_is_deterministic():
+    di = small("ragged_b64_1k_16k", lengths=[900, 3000, 17, 5000])
+    outs = [run_gva(di)[0] for _ in range(5)]
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0])
+
+
+def test_decode_flags_slots_outside_cache():
+    """A sequence that reaches past the cache is flagged in the status word;
+    missing rows read as zeros and nothing faults."""
+    di = small("350m_b8_t4096", lengths=[40, 40])
+    di.seq_offset = torch.tensor([0, di.num_slots - 10], dtype=torch.int32)
+    for flags in (0, gva.FLAG_FMA_PATH):
+        out, _, _, st = run_gva(di, flags=flags)
+        assert st & gva.DEVERR_RANGE
+        assert np.all(np.isfinite(out))
+
+
+# ------------------------------------------------------------------ GQA comparison kernel
+
+@pytest.mark.parametrize("flags", [0, gva.FLAG_FMA_PATH], ids=["tensor", "fma"])
+@pytest.mark.parametrize("name", ["350m_b8_t4096", "dr24_b4_t32768", "d128_b1_t131072"])
+def test_gqa_matches_oracle(name, flags):
+    wl = WORKLOADS[name]
+    gi = make_gqa_inputs(wl, extra_slots=1, lengths=np.array([1, 33, 500, 1025]))
+    out, lse, st = run_gqa(gi, wl.H, wl.G, wl.d_h, wl.torch_dtype, flags=flags)
+    ref, ref_lse = oracle_gqa(gi)
+    assert st == 0
+    assert_close(out, ref, wl.dtype, name)
+    lse_close(lse, ref_lse)
+
+
+def test_shared_kv_gva_equals_gqa():
+    """M_h = I and d_r = 0 turn GVA into attention with K = V: the GVA kernels
+    and the GQA kernel (given K_cache = V_cache) agree with each other and with
+    the oracle."""
+    wl = WORKLOADS["350m_b8_t4096"].scaled(d_n=64, d_r=0)
+    di = make_decode_inputs(wl, extra_slots=0, lengths=np.array([300, 1, 1000]))
+    di.M = torch.eye(64, dtype=torch.bfloat16).expand(16, 64, 64).contiguous()
+    out_gva, lse_gva, _, _ = run_gva(di)
+    ref, ref_lse = oracle_gva(di)
+    assert_close(out_gva, ref, "bf16", "gva K=V")
+    # GQA with q = the absorbed query (identity map: q itself), K = V
+    from compressed_kv_cache_gva_b200.synth import GQAInputs
+    gi = GQAInputs(seq_len=di.seq_len, seq_offset=di.seq_offset, q=di.q, K=di.V, V=di.V,
+                   num_slots=di.num_slots)
+    out_gqa, lse_gqa, _ = run_gqa(gi, 16, 4, 64, torch.bfloat16)
+    assert_close(out_gqa, ref, "bf16", "gqa K=V")
+    assert np.max(np.abs(out_gqa - out_gva)) < 1e-3
