@@ -1,0 +1,471 @@
+"""Benchmark of one GVA decode step on synthetic caches.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole decode path over one batch: absorb the queries
+(q M^T + query RoPE), append each sequence's new token (value copy + rotated
+positional key), then decode attention over the history plus the new token.
+Every step reads a different copy of the cache (copies rotate; together they
+exceed 3x the L2), so no step starts with its cache in L2.
+
+Printed: ONE JSON line on rank 0.  value = cache GB/s of the whole job (algorithmic
+cache bytes of all steps on all ranks / max-over-ranks device time).  Under
+torchrun every rank runs its own batch (weak scaling, no collective on the data
+path).  `--impl reference` times the float64 CPU oracle on the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from compressed_kv_cache_gva_b200 import gva  # noqa: E402
+from compressed_kv_cache_gva_b200.synth import (WORKLOADS, make_append_inputs,  # noqa: E402
+                                                make_decode_inputs, make_gqa_inputs)
+
+METRIC = "GVA decode cache GB/s & %HBM peak (1xB200); decode steps/s vs same-shape GQA"
+DEFAULT_WORKLOAD = "350m_b8_t4096"
+L2_BYTES = 126 * 1024 * 1024
+NOMINAL_HBM_GBS = 8000.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20000)
+    p.add_argument("--warmup", type=int, default=200)
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--fma", action="store_true", help="decode on the CUDA-core FMA path")
+    p.add_argument("--ctas-per-sm", type=int, default=0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    return p.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms in a thread."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.samples = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.index), "-lms", "50"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 10:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        win = [s for t, s in self.samples if t0 <= t <= t1]
+        label = "timed"
+        if len(win) < 3:
+            return None
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return float("nan")
+        sm = [num(s[2]) for s in win]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for s in win:
+            for n, v in zip(names, s[6:10]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.nanmedian(sm)), "sm_max_mhz": num(win[0][3]),
+                "reasons": sorted(reasons), "samples": len(win), "window": label,
+                "power_w_median": float(np.nanmedian([num(s[4]) for s in win]))}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def cache_row_bytes(wl):
+    return (wl.G * wl.d_h + wl.d_r) * wl.elem_bytes
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "compressed_kv_cache_gva_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[workload][kernel_key]
+        if e.get("source_hash") != kernel_source_hash():
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def run_ours(args, rank, world, local):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = WORKLOADS[args.workload].scaled(seed=WORKLOADS[args.workload].seed + rank)
+    di = make_decode_inputs(wl, extra_slots=1)
+    B, H, G, d_h, d_r = len(di.seq_len), wl.H, wl.G, wl.d_h, wl.d_r
+    L = di.seq_len.numpy().astype(np.int64)
+    row_bytes = cache_row_bytes(wl)
+    step_tokens = int((L + 1).sum())                       # history + the appended token
+    step_cache_bytes = step_tokens * row_bytes
+    cache_bytes = di.num_slots * row_bytes
+    R = max(2, math.ceil(3 * L2_BYTES / cache_bytes))
+    flags = gva.FLAG_FMA_PATH if args.fma else 0
+    sh = gva.make_shape(B, H, G, d_h, wl.d_n, d_r, cache_dtype=wl.torch_dtype, rope_base=wl.rope_base,
+                        flags=flags, ctas_per_sm=args.ctas_per_sm)
+
+    d = lambda t: t.to(dev).contiguous()
+    Vs = [d(di.V) for _ in range(R)]
+    KRs = [d(di.k_rope) for _ in range(R)]
+    q, M = d(di.q), d(di.M)
+    soff = d(di.seq_offset)
+    slen_step = d(torch.from_numpy((L + 1).astype(np.int32)))
+    qpos = d(di.seq_len)                                    # new token at position L_b
+    slots_np = (di.seq_offset.numpy() + L).astype(np.int32)
+    ap = make_append_inputs(wl, slots_np, L.astype(np.int32), seed=7 + rank)
+    v_new, kpe_new, slot, pos = d(ap.v_new), d(ap.kpe_new), d(ap.slot), d(ap.pos)
+    q_abs = torch.empty(B, H, d_h + d_r, dtype=torch.float32, device=dev)
+    out = torch.empty(B, H, d_h, dtype=torch.float32, device=dev)
+    max_total = step_tokens
+    ws = gva.new_workspace(sh, max_total, device=dev)
+
+    def step(c):
+        gva.absorb_query(sh, q, M, qpos, q_abs)
+        gva.append_cache(sh, v_new, kpe_new, slot, pos, Vs[c], KRs[c])
+        gva.decode_attention(sh, q_abs, Vs[c], KRs[c], soff, slen_step, max_total, out, None, ws)
+
+    def decode_only(c):
+        gva.decode_attention(sh, q_abs, Vs[c], KRs[c], soff, slen_step, max_total, out, None, ws)
+
+    # eager warm-up (initialises the library and the launch attributes)
+    for c in range(R):
+        step(c)
+    torch.cuda.synchronize()
+
+    def capture(fn, n, first=0):
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                for i in range(n):
+                    fn((first + i) % R)
+        torch.cuda.current_stream().wait_stream(s)
+        return g
+
+    CHUNK = 256
+
+    def graphs_for(fn, K):
+        gs = []
+        done = 0
+        while done < K:
+            n = min(CHUNK, K - done)
+            gs.append((capture(fn, n, done), n))
+            done += n
+        return gs
+
+    def replay(gs):
+        for g, _ in gs:
+            g.replay()
+
+    def timed(gs, K, sampler_window=None):
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        st = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0 = time.time()
+        e0.record(st)
+        replay(gs)
+        e1.record(st)
+        torch.cuda.synchronize()
+        t1 = time.time()
+        if world > 1:
+            torch.distributed.barrier()
+        ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms, t0, t1
+
+    K, W = args.steps, args.warmup
+    g_warm = graphs_for(step, max(W, 1))
+    g_time = graphs_for(step, K)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.2)
+    tw0 = time.time()
+    replay(g_warm)
+    torch.cuda.synchronize()
+    ms, t0, t1 = timed(g_time, K)
+    clocks = sampler.summary(tw0, t1)
+    if clocks is None:
+        # timed region too short for 50 ms sampling: keep the same graphs running
+        # (untimed) for about a second and report the clocks seen under that load
+        s0 = time.time()
+        while time.time() - s0 < 1.2:
+            replay(g_time)
+            torch.cuda.synchronize()
+        clocks = sampler.summary(tw0, time.time())
+        if clocks is not None:
+            clocks["window"] = "warm-up + timed + untimed soak of the same step graphs"
+    sampler.stop()
+    assert gva.workspace_status(ws) == 0, "device status word set"
+
+    # decode-only timing (roofline of the dominant kernel) and the GQA comparison
+    g_dec = graphs_for(decode_only, K)
+    replay(g_dec)
+    ms_dec, _, _ = timed(g_dec, K)
+    gi = make_gqa_inputs(wl, extra_slots=1)
+    Kq = [d(gi.K) for _ in range(R)]
+    Vq = [d(gi.V) for _ in range(R)]
+    sh_q = gva.make_shape(B, H, G, d_h, d_h, 0, cache_dtype=wl.torch_dtype, flags=flags,
+                          ctas_per_sm=args.ctas_per_sm)
+    qg = d(gi.q)
+    slen_q = d(torch.from_numpy((gi.seq_len.numpy() + 1).astype(np.int32)))
+    soff_q = d(gi.seq_offset)
+    tot_q = int(gi.seq_len.numpy().astype(np.int64).sum()) + B
+    ws_q = gva.new_workspace(sh_q, tot_q, device=dev)
+    out_q = torch.empty(B, H, d_h, dtype=torch.float32, device=dev)
+
+    def gqa_decode(c):
+        gva.gqa_decode_attention(sh_q, qg, Kq[c], Vq[c], soff_q, slen_q, tot_q, out_q, None, ws_q)
+
+    for c in range(R):
+        gqa_decode(c)
+    g_gqa = graphs_for(gqa_decode, K)
+    replay(g_gqa)
+    ms_gqa, _, _ = timed(g_gqa, K)
+    gqa_bytes = tot_q * 2 * G * d_h * wl.elem_bytes
+    del Kq, Vq
+
+    # end to end through the public API with host buffers: every step copies its
+    # inputs (q, new value, new positional key, slot, position) from pinned host
+    # memory and reads the output back to pinned host memory
+    h_in = [t.pin_memory() for t in (di.q, ap.v_new, ap.kpe_new, ap.slot, ap.pos)]
+    d_in = [q, v_new, kpe_new, slot, pos]
+    h_out = torch.empty(B, H, d_h, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step(c):
+        for hd, dd in zip(h_in, d_in):
+            dd.copy_(hd, non_blocking=True)
+        step(c)
+        h_out.copy_(out, non_blocking=True)
+
+    g_e2e = graphs_for(e2e_step, K)
+    replay(g_e2e)
+    ms_e2e, _, _ = timed(g_e2e, K)
+
+    hbm_peak, peak_kind = load_peaks()
+    ms_step = ms / K
+    value = world * K * step_cache_bytes / (ms * 1e-3) / 1e9
+    dec_s = ms_dec / K * 1e-3
+    alg_dec_bytes = step_cache_bytes + B * H * (d_h + d_r) * 4 + B * H * d_h * 4
+    achieved = alg_dec_bytes / dec_s / 1e9
+    kernel_key = "decode_simt_kernel" if args.fma else "decode_mma_kernel"
+    res = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": round(ms_step, 6), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "B": B, "H": H, "G": G, "d_h": d_h, "d_n": wl.d_n, "d_r": d_r,
+                   "T": wl.T, "ragged": wl.ragged, "rope_base": wl.rope_base,
+                   "tokens_per_step": step_tokens, "cache_bytes_per_step": step_cache_bytes,
+                   "l2": f"inputs larger than L2: {R} rotating cache copies, "
+                         f"{R * cache_bytes / 2**20:.0f} MiB",
+                   "parallelism": f"weak: {world} independent batch(es), one per GPU",
+                   "step": "absorb + append + decode (split + combine)", "graphs": "CUDA graphs",
+                   "decode_path": "fma" if args.fma else "tensor"},
+        "steps_per_s": round(world * K / (ms * 1e-3), 1),
+        "pct_hbm_peak": {"of_measured": round(value / world / hbm_peak, 4),
+                         "of_nominal_8TBs": round(value / world / NOMINAL_HBM_GBS, 4)},
+        "gqa_comparison": {
+            "gva_decode_steps_per_s": round(K / (ms_dec * 1e-3), 1),
+            "gqa_decode_steps_per_s": round(K / (ms_gqa * 1e-3), 1),
+            "decode_speedup_vs_gqa": round(ms_gqa / ms_dec, 4),
+            "gva_cache_bytes": step_cache_bytes, "gqa_cache_bytes": gqa_bytes,
+            "cache_ratio": round(step_cache_bytes / gqa_bytes, 6),
+            "gqa_cache_GBs": round(gqa_bytes / (ms_gqa / K * 1e-3) / 1e9, 2)},
+        "roofline": {"bound": "hbm", "kernel": f"{kernel_key} + combine (one gva_decode_attention call)",
+                     "achieved": round(achieved, 2), "peak": hbm_peak, "peak_kind": peak_kind,
+                     "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                     "alg_bytes_per_launch": alg_dec_bytes, "us_per_launch": round(dec_s * 1e6, 3),
+                     "traffic": ncu_traffic(kernel_key, wl.name)},
+        "e2e": {"value": round(world * K * step_cache_bytes / (ms_e2e * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(ms_e2e / K, 6)},
+        "gpu_launches": 4 * K,
+        "clocks": clocks,
+    }
+    return res, di
+
+
+# ----------------------------------------------------------------------------- oracle arm
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle(wl, di, budget_s, max_units=None):
+    """Oracle decode on (sequence, head) pairs until the time budget is spent.
+    Returns (cache bytes attended per second, description)."""
+    import oracle
+    from compressed_kv_cache_gva_b200.synth import as_f64
+    q, M = as_f64(di.q), as_f64(di.M)
+    V, KR = as_f64(di.V), as_f64(di.k_rope)
+    L = di.seq_len.numpy()
+    pairs = [(b, h) for b in range(len(L)) for h in range(wl.H)]
+    done, nbytes = 0, 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s and (max_units is None or done < max_units):
+        b, h = pairs[done % len(pairs)]
+        oracle.gva_decode(q, M, di.q_pos.numpy(), V, KR, di.seq_offset.numpy(), L, wl.d_n, wl.d_r,
+                          wl.rope_base, pairs=[(b, h)])
+        # one (b, h) pair attends L_b rows; H pairs of a sequence cover its whole cache row
+        nbytes += int(L[b]) * cache_row_bytes(wl) / wl.H
+        done += 1
+    dt = time.perf_counter() - t0
+    return nbytes / dt / 1e9, f"{done} (sequence, head) pairs of the full-size cache, {dt:.1f} s", dt, done
+
+
+def cpu_baseline(wl, di, seconds):
+    gbs, desc, dt, n = time_oracle(wl, di, seconds)
+    return {"value": round(gbs, 6), "unit": "GB/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": desc}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    wl = WORKLOADS[args.workload]
+    di = make_decode_inputs(wl, extra_slots=1)
+    total_steps = args.steps + args.warmup
+    per_step = max(0.002, min(2.0, 150.0 / total_steps))
+    import oracle  # noqa: F401
+    for _ in range(args.warmup):
+        time_oracle(wl, di, per_step, max_units=1)
+    t0 = time.perf_counter()
+    nbytes_rate = []
+    for _ in range(args.steps):
+        g, _, dt, n = time_oracle(wl, di, per_step, max_units=None if per_step > 0.01 else 1)
+        nbytes_rate.append((g, dt))
+    elapsed = time.perf_counter() - t0
+    total_bytes = sum(g * 1e9 * dt for g, dt in nbytes_rate)
+    value = total_bytes / elapsed / 1e9
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(elapsed / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "step": "float64 CPU oracle, non-absorbed route, "
+                                                  "bounded sample of (sequence, head) pairs per step"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": oracle_threads(),
+                         "kind": "oracle",
+                         "sample": f"each step: oracle decode of (sequence, head) pairs for "
+                                   f"~{per_step * 1e3:.0f} ms"},
+        "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    res, di = run_ours(args, rank, world, local)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        wl = WORKLOADS[args.workload]
+        res["cpu_baseline"] = cpu_baseline(wl, di, args.cpu_seconds)
+    elif rank == 0:
+        res["cpu_baseline"] = None
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

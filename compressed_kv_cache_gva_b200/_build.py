@@ -43,14 +43,17 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, extra_flags=(), out: str = LIB) -> str:
+    """Compile every csrc/*.cu and link them into `out` (default: the package's
+    libgva.so).  `extra_flags` go to every nvcc compile (e.g. -DGVA_TRACE)."""
+    if not force and not extra_flags and out == LIB and up_to_date():
         return LIB
     os.makedirs(OBJDIR, exist_ok=True)
     srcs = _sources()
 
+    tag = "" if not extra_flags else "_" + str(abs(hash(tuple(extra_flags))))
     def compile_one(src):
-        obj = os.path.join(OBJDIR, os.path.basename(src) + ".o")
+        obj = os.path.join(OBJDIR, os.path.basename(src) + tag + ".o")
         cmd = [NVCC, *FLAGS, *extra_flags, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
@@ -61,16 +64,22 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
 
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
         objs = list(ex.map(compile_one, srcs))
-    tmp = LIB + ".tmp"
+    tmp = out + ".tmp"
     cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart", "static",
            *objs, "-o", tmp]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
-    extra = [a for a in sys.argv[1:] if a.startswith("-X") or a.startswith("--resource")]
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, extra_flags=extra))
+    import argparse
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("-v", action="store_true")
+    ap.add_argument("--trace", action="store_true", help="build with -DGVA_TRACE")
+    ap.add_argument("--out", default=LIB)
+    a = ap.parse_args()
+    print(build(force=a.force, verbose=a.v, extra_flags=["-DGVA_TRACE"] if a.trace else [], out=a.out))

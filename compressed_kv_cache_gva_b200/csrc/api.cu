@@ -12,6 +12,9 @@
 namespace {
 
 thread_local char g_err[320] = "";
+#ifdef GVA_TRACE
+unsigned long long* g_trace = nullptr;
+#endif
 
 gva_status_t fail(gva_status_t s, const char* fmt, ...) {
   va_list ap;
@@ -55,8 +58,9 @@ gva_status_t check_shape(const gva_shape_t* sh, bool gqa) {
   if (sh->d_h < 1 || sh->d_h > 512) return fail(GVA_ERR_INVALID_ARG, "d_h=%d outside [1,512]", sh->d_h);
   if (!gqa) {
     if (sh->d_n < 0 || sh->d_n > 1024) return fail(GVA_ERR_INVALID_ARG, "d_n=%d outside [0,1024]", sh->d_n);
-    if (sh->d_r < 0 || sh->d_r > 256 || (sh->d_r & 1))
-      return fail(GVA_ERR_INVALID_ARG, "d_r=%d must be even and in [0,256]", sh->d_r);
+    if (sh->d_r < 0 || sh->d_r > 2 * gva::kMaxRopePairs || (sh->d_r & 1))
+      return fail(GVA_ERR_INVALID_ARG, "d_r=%d must be even and in [0,%d]", sh->d_r,
+                  2 * gva::kMaxRopePairs);
     if (!(sh->rope_base > 0.0) || !isfinite(sh->rope_base))
       return fail(GVA_ERR_INVALID_ARG, "rope_base must be positive and finite");
   }
@@ -176,6 +180,9 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
   a.part_ml = reinterpret_cast<float2*>(ws + p.ws.ml_off);
   a.part_o = reinterpret_cast<float*>(ws + p.ws.o_off);
   a.grid = p.grid;
+#ifdef GVA_TRACE
+  a.trace = g_trace;
+#endif
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   cudaError_t err;
@@ -226,6 +233,12 @@ const char* gva_status_string(gva_status_t s) {
 
 const char* gva_last_error(void) { return g_err; }
 
+#ifdef GVA_TRACE
+// Trace builds only: device buffer of grid * 8 uint64 receiving the timeline of
+// the next split kernels (NULL turns tracing off).
+void gva_trace_set_buffer(void* dev_buf) { g_trace = static_cast<unsigned long long*>(dev_buf); }
+#endif
+
 gva_status_t gva_absorb_query(const gva_shape_t* shp, const void* q, const void* M,
                               const int32_t* q_pos, float* q_abs, void* stream) {
   gva_status_t s = check_shape(shp, false);
@@ -236,7 +249,7 @@ gva_status_t gva_absorb_query(const gva_shape_t* shp, const void* q, const void*
     return fail(GVA_ERR_INVALID_ARG, "a required pointer is NULL");
   if (!aligned16(q) || (M && !aligned16(M)) || !aligned16(q_pos) || !aligned16(q_abs))
     return fail(GVA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
-  const size_t smem = sizeof(float) * ((size_t)sh.d_h * (sh.d_n + 1) + sh.d_n + sh.d_r);
+  const size_t smem = gva::absorb_smem_bytes(sh);
   if (smem > 200 * 1024) return fail(GVA_ERR_UNSUPPORTED, "M_h too large for one CTA (%zu bytes)", smem);
   const float c = scale_of(sh, false) * gva::kLog2e;
   cudaError_t e = gva::launch_absorb(sh, q, M, q_pos, q_abs, c, static_cast<cudaStream_t>(stream));

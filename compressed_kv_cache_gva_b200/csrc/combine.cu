@@ -4,55 +4,150 @@
 //   m* = max_c m_c,  L = sum_c 2^(m_c - m*) l_c,  out = sum_c 2^(m_c - m*) o_c / L,
 //   lse = (m* + log2 L) * ln 2  (natural log of sum_j exp(s_j)).
 // The merge order is fixed by piece index, so results do not depend on which CTA
-// finished first.  One CTA per (sequence, block of heads); one thread per output
-// element.
+// finished first.
 #include "common.cuh"
 #include "launch.h"
 
 namespace gva {
 
+constexpr int kCombineScanMaxB = 64;   // batches up to this size find their pieces
+                                        // from the lengths before waiting
+constexpr int kCombinePieces = 8;       // pieces per thread requested at once
+
+// grid (B, H, ceil(d_h / 32)); block = 32 output columns x PG piece groups.
+// Thread (pg, lane) merges pieces pg, pg+PG, ... of column d = 32*z + lane with
+// its own running max; all its loads are requested before the first merge.  The
+// PG running states are then merged through shared memory.  For small batches
+// the piece range of sequence b is recomputed from the lengths (caller input)
+// before waiting on the split kernel, so that after the wait only the partials
+// are read.
 template <typename TO>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(1024)
     combine_kernel(const DecodeArgs a, TO* __restrict__ out, float* __restrict__ lse) {
-  const int b = blockIdx.x;
-  const int d_h = a.d_h, H = a.H;
-  const int hpb = d_h >= 128 ? 1 : 128 / d_h;
-  if (d_h < 128 && (int)threadIdx.x >= hpb * d_h) return;
-  const int h = blockIdx.y * hpb + (d_h >= 128 ? 0 : threadIdx.x / d_h);
-  if (h >= H) return;
-  const int2 meta = a.meta[b];
-  const int base = meta.x, n = meta.y;
-  float mx = -INFINITY;
-  for (int c = 0; c < n; ++c) mx = fmaxf(mx, a.part_ml[(size_t)(base + c) * H + h].x);
-  float wsum = 0.f;
-  for (int c = 0; c < n; ++c) {
-    const float2 ml = a.part_ml[(size_t)(base + c) * H + h];
-    wsum += ex2(ml.x - mx) * ml.y;
-  }
-  const float inv = n > 0 ? 1.f / wsum : 0.f;
-  const int dstep = d_h >= 128 ? 128 : d_h;
-  for (int d = (d_h >= 128 ? threadIdx.x : threadIdx.x % d_h); d < d_h; d += dstep) {
-    float acc = 0.f;
-    for (int c = 0; c < n; ++c) {
-      const float w = ex2(a.part_ml[(size_t)(base + c) * H + h].x - mx);
-      acc = fmaf(w, a.part_o[((size_t)(base + c) * H + h) * d_h + d], acc);
+  __shared__ float sm_m[32][33], sm_l[32][33], sm_o[32][33];
+  __shared__ int s_meta[2];
+  const int b = blockIdx.x, h = blockIdx.y, d = blockIdx.z * 32 + (threadIdx.x & 31);
+  const int H = a.H, d_h = a.d_h;
+  const int tid = threadIdx.x, lane = tid & 31, pg = tid >> 5, npg = blockDim.x >> 5;
+  const bool scan = a.B <= kCombineScanMaxB;
+  if (scan && pg == 0) {
+    // lengths of sequences < b, of b, and of the whole batch (one warp)
+    long long before = 0, total = 0;
+    int Lb = 0;
+    for (int j = lane; j < a.B; j += 32) {
+      const int L = max(__ldg(a.seq_len + j), 0);
+      total += L;
+      if (j < b) before += L;
+      if (j == b) Lb = L;
     }
-    const float v = acc * inv;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      before += __shfl_xor_sync(0xffffffffu, before, o);
+      total += __shfl_xor_sync(0xffffffffu, total, o);
+      Lb += __shfl_xor_sync(0xffffffffu, Lb, o);
+    }
+    if (lane == 0) {
+      int first = 0, count = 0;
+      if (Lb > 0 && total < (1ll << 31)) {
+        const int per = (int)((total + a.grid - 1) / a.grid);
+        const int span = max(a.tile, (per + a.tile - 1) / a.tile * a.tile);
+        const int f = (int)(before / span), l = (int)((before + Lb - 1) / span);
+        first = f + b;
+        count = l - f + 1;
+      }
+      s_meta[0] = first;
+      s_meta[1] = count;
+    }
+  }
+  pdl_wait();
+  pdl_trigger();
+#ifdef GVA_TRACE
+  const int cid = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+  if (a.trace && tid == 0 && cid < 16384) {
+    unsigned long long tt;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(tt));
+    a.trace[4096 * 8 + cid * 2] = tt;
+  }
+#endif
+  int base, n;
+  if (scan) {
+    __syncthreads();
+    base = s_meta[0];
+    n = s_meta[1];
+  } else {
+    const int2 meta = a.meta[b];
+    base = meta.x;
+    n = meta.y;
+  }
+  const bool col = d < d_h;
+  const float2* ml = a.part_ml + (size_t)base * H + h;
+  const float* po = a.part_o + ((size_t)base * H + h) * d_h + (col ? d : 0);
+  const size_t mstride = H, ostride = (size_t)H * d_h;
+  float m = -INFINITY, l = 0.f, o = 0.f;
+  for (int c0 = pg; c0 < n; c0 += kCombinePieces * npg) {
+    float2 e[kCombinePieces];
+    float x[kCombinePieces];
+#pragma unroll
+    for (int u = 0; u < kCombinePieces; ++u) {
+      const int c = c0 + u * npg;
+      if (c < n) {
+        e[u] = ml[(size_t)c * mstride];
+        x[u] = po[(size_t)c * ostride];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kCombinePieces; ++u) {
+      if (c0 + u * npg >= n) break;
+      const float mn = fmaxf(m, e[u].x);
+      const float f = ex2(m - mn), w = ex2(e[u].x - mn);
+      l = l * f + w * e[u].y;
+      o = o * f + w * x[u];
+      m = mn;
+    }
+  }
+  sm_m[pg][lane] = m;
+  sm_l[pg][lane] = l;
+  sm_o[pg][lane] = o;
+  __syncthreads();
+  if (pg != 0) return;
+  float M = -INFINITY;
+  for (int u = 0; u < npg; ++u) M = fmaxf(M, sm_m[u][lane]);
+  float L = 0.f, O = 0.f;
+  for (int u = 0; u < npg; ++u) {
+    const float mu = sm_m[u][lane];
+    if (mu == -INFINITY) continue;                 // a group that saw no piece
+    const float f = ex2(mu - M);
+    L = fmaf(f, sm_l[u][lane], L);
+    O = fmaf(f, sm_o[u][lane], O);
+  }
+  if (col) {
+    const float v = n > 0 ? O / L : 0.f;
     if constexpr (sizeof(TO) == 2) out[((size_t)b * H + h) * d_h + d] = __float2bfloat16_rn(v);
     else out[((size_t)b * H + h) * d_h + d] = v;
-    if (d == 0 && lse) lse[(size_t)b * H + h] = n > 0 ? (mx + log2f(wsum)) * kLn2 : -INFINITY;
   }
+  if (lane == 0 && blockIdx.z == 0 && lse)
+    lse[(size_t)b * H + h] = n > 0 ? (M + log2f(L)) * kLn2 : -INFINITY;
+#ifdef GVA_TRACE
+  if (a.trace && tid == 0 && cid < 16384) {
+    unsigned long long tt;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(tt));
+    a.trace[4096 * 8 + cid * 2 + 1] = tt;
+  }
+#endif
 }
 
 cudaError_t launch_combine(const gva_shape_t& sh, const DecodeArgs& a, void* out, float* lse,
                            cudaStream_t st) {
-  const int hpb = sh.d_h >= 128 ? 1 : 128 / sh.d_h;
-  dim3 grid(sh.B, (sh.H + hpb - 1) / hpb);
+  const dim3 grid(sh.B, sh.H, (sh.d_h + 31) / 32);
+  // a sequence has about grid/B + 1 pieces (ragged batches: more for the long
+  // ones); aim at ~kCombinePieces pieces per thread, 1..32 piece groups
+  const int per_seq = a.grid / (sh.B > 0 ? sh.B : 1) + 2;
+  int npg = (per_seq + kCombinePieces - 1) / kCombinePieces;
+  npg = npg < 1 ? 1 : (npg > 32 ? 32 : npg);
   if (sh.out_dtype == GVA_BF16)
-    combine_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(a, (__nv_bfloat16*)out, lse);
-  else
-    combine_kernel<float><<<grid, 128, 0, st>>>(a, (float*)out, lse);
-  return cudaGetLastError();
+    return launch_pdl(combine_kernel<__nv_bfloat16>, grid, dim3(32 * npg), 0, st, a,
+                      (__nv_bfloat16*)out, lse);
+  return launch_pdl(combine_kernel<float>, grid, dim3(32 * npg), 0, st, a, (float*)out, lse);
 }
 
 }  // namespace gva

@@ -58,7 +58,23 @@ struct DecodeArgs {
   float* part_o;             // [P][H][d_h] un-normalised output
   int grid;                  // CTAs of the split kernel
   int tile;                  // span granularity in tokens
+  unsigned long long* trace; // per-CTA timestamps, only with -DGVA_TRACE (else unused)
 };
+
+// Optional timeline instrumentation: with -DGVA_TRACE each CTA of the split kernel
+// stores %globaltimer (ns) at fixed points of its life into trace[cta * 8 + slot].
+__device__ __forceinline__ void trace_mark(const DecodeArgs& a, int slot) {
+#ifdef GVA_TRACE
+  if (a.trace) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    a.trace[blockIdx.x * 8 + slot] = t;
+  }
+#else
+  (void)a;
+  (void)slot;
+#endif
+}
 
 // ---------------------------------------------------------------------------
 // Split-KV work list.  Tokens of all sequences are concatenated in batch order;
@@ -149,6 +165,25 @@ __device__ inline void write_meta(const DecodeArgs& a, const int* prefix, Span s
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel here runs a prologue that reads
+// nothing the preceding kernel of the stream writes, then waits for that kernel
+// (griddepcontrol.wait: it has completed and its writes are visible), then lets
+// the next kernel start launching.  Since every kernel waits before it triggers,
+// a kernel can only start once the kernel two places earlier has completed, so
+// the chain stays ordered transitively.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// RoPE inverse frequencies base^(-2i/d_r), evaluated in float64 on the host.
+constexpr int kMaxRopePairs = 64;
+struct RopeTable {
+  double inv_freq[kMaxRopePairs];
+};
+
+// ---------------------------------------------------------------------------
 // Small numeric helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float ex2(float x) {  // 2^x on the SFU (PTX ex2.approx)
@@ -225,6 +260,27 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
+}
+
+// Same, with an L2 eviction-priority policy (from createpolicy) for data read once.
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                                 uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// Barrier among `count` threads (a multiple of 32) of the CTA, id 1..15.
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -13,8 +13,7 @@ cudaError_t run(const gva_shape_t& sh, DecodeArgs& a, const CUtensorMap& tx, con
   auto k = decode_mma_kernel<C>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<a.grid, C::THREADS, smem, st>>>(a, tx, tv, tk);
-  return cudaGetLastError();
+  return launch_pdl(k, dim3(a.grid), dim3(C::THREADS), smem, st, a, tx, tv, tk);
 }
 
 // Visit the instantiation matching (d_h, G, H/G, padded d_r, gqa); f receives a

@@ -24,12 +24,15 @@
 
 namespace gva {
 
-template <int D_H_, int NG_, int HPG_, int DRP_, bool GQA_>
+template <int D_H_, int NG_, int HPG_, int DRP_, bool GQA_, int W_ = 1>
 struct MmaCfg {
   static constexpr int D_H = D_H_, NG = NG_, HPG = HPG_, DRP = GQA_ ? 0 : DRP_;
   static constexpr bool GQA = GQA_;
   static constexpr int ROW_BYTES = NG * D_H * 2 * (GQA ? 2 : 1);
-  static constexpr int TT_RAW = 16384 / ROW_BYTES;
+#ifndef GVA_TILE_BYTES   // bytes of cache rows per pipeline stage (tuning knob)
+#define GVA_TILE_BYTES 16384
+#endif
+  static constexpr int TT_RAW = (GQA ? 2 * GVA_TILE_BYTES : GVA_TILE_BYTES) / ROW_BYTES;
   static constexpr int TT = TT_RAW >= 64 ? 64 : (TT_RAW >= 32 ? 32 : 16);   // tokens per tile
   static constexpr int CB = D_H / 64;                 // 64-column boxes per group
   static constexpr int BOX = TT * 128;                // bytes of one [TT x 64] bf16 box
@@ -37,52 +40,70 @@ struct MmaCfg {
   static constexpr int VB = GQA ? XB : 0;             // separate value tile (GQA)
   static constexpr int KRB = DRP ? TT * DRP * 2 : 0;  // positional key tile
   static constexpr int STAGE = XB + VB + (KRB + 1023) / 1024 * 1024;
-  static constexpr int STAGES_RAW = (96 * 1024) / STAGE;
+#ifndef GVA_PIPE_BYTES   // shared memory of the stage ring per CTA (tuning knob)
+#define GVA_PIPE_BYTES (96 * 1024)
+#endif
+  static constexpr int STAGES_RAW = GVA_PIPE_BYTES / STAGE;
   static constexpr int STAGES = STAGES_RAW < 2 ? 2 : (STAGES_RAW > 12 ? 12 : STAGES_RAW);
   static constexpr int PIPE = STAGES * STAGE;
   static constexpr uint32_t TX = XB + VB + KRB;       // bytes TMA delivers per stage
-  static constexpr int THREADS = (NG + 1) * 32;
+  static constexpr int MT = TT / 16;                  // 16-token m-tiles per tile
+  static constexpr int W = W_ < MT ? W_ : MT;         // consumer warps per group
+  static constexpr int MW = MT / W;                   // m-tiles per consumer warp
+  static constexpr int NCW = NG * W;                  // consumer warps
+  static constexpr int THREADS = (NCW + 1) * 32;
   static constexpr int NT = HPG == 8 ? 2 : 1;         // 8-column MMA tiles
   static constexpr int KS = D_H / 16;                 // content k-steps (= d m-tiles)
   static constexpr int RS = DRP / 16;                 // positional k-steps
-  static constexpr int MT = TT / 16;                  // 16-token m-tiles per tile
+  // end-of-piece merge of the W warps of a group: (m, l) per warp and lane quad,
+  // and the output fragments of warps 1..W-1
+  static constexpr int MERGE_ML = W * 4 * 4;                    // floats per group
+  static constexpr int MERGE_O = (W - 1) * 32 * NT * KS * 4;   // floats per group
+  static constexpr int MERGE = W > 1 ? NG * (MERGE_ML + MERGE_O) * 4 : 0;  // bytes
   static constexpr int KR_SW = DRP * 2;               // swizzle span of the k_rope box
   static_assert(HPG == 4 || HPG == 8, "heads per group");
   static_assert(D_H % 64 == 0, "d_h");
   static_assert(DRP == 0 || DRP == 16 || DRP == 32, "padded d_r");
 
   static size_t smem_bytes(int B) {
-    return 1024 + PIPE + 16 * STAGES + sizeof(int) * (B + 1) + 16 + sizeof(long long) * 33;
+    return 1024 + PIPE + MERGE + 16 * STAGES + 2 * sizeof(int) * (B + 1) + 16 +
+           sizeof(long long) * 33;
   }
 };
 
 template <class C>
-__global__ void __launch_bounds__(C::THREADS)
+__global__ void __launch_bounds__(C::THREADS, 2)
     decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_x,
                       const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_kr) {
   extern __shared__ unsigned char smraw[];
   uint8_t* pipe = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(pipe + C::PIPE);
+  float* merge = reinterpret_cast<float*>(pipe + C::PIPE);
+  uint64_t* full = reinterpret_cast<uint64_t*>(pipe + C::PIPE + C::MERGE);
   uint64_t* empty = full + C::STAGES;
   int* prefix = reinterpret_cast<int*>(empty + C::STAGES);
+  int* offs = prefix + a.B + 1;
   long long* wtmp = reinterpret_cast<long long*>(
-      (reinterpret_cast<uintptr_t>(prefix + a.B + 1) + 15) & ~uintptr_t(15));
+      (reinterpret_cast<uintptr_t>(offs + a.B + 1) + 15) & ~uintptr_t(15));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) trace_mark(a, 0);
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(smem_u32(full + s), 1);
-      mbar_init(smem_u32(empty + s), C::NG);
+      mbar_init(smem_u32(empty + s), C::NCW);
     }
     fence_barrier_init();
   }
-  if (warp == C::NG && lane == 0) {
+  if (warp == C::NCW && lane == 0) {
     prefetch_tmap(&tm_x);
     if (C::GQA) prefetch_tmap(&tm_v);
     if (C::DRP) prefetch_tmap(&tm_kr);
   }
+  // The lengths and offsets are caller inputs that no kernel of this library
+  // writes, so they are read before waiting on the preceding kernel.
+  for (int b = threadIdx.x; b < a.B; b += blockDim.x) offs[b] = __ldg(a.seq_offset + b);
   long long total64 = block_scan_lengths(a.seq_len, a.B, prefix, wtmp);   // syncs the block
   int total = (int)total64;
   if (total64 >= (1ll << 31)) {
@@ -90,6 +111,9 @@ __global__ void __launch_bounds__(C::THREADS)
     total = 0;
   }
   const Span sp = make_span(total, gridDim.x, C::TT);
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x == 0) trace_mark(a, 1);
   if (blockIdx.x == 0) write_meta(a, prefix, sp);
   const int s0 = blockIdx.x * sp.span;
   if (s0 >= total) return;
@@ -97,13 +121,17 @@ __global__ void __launch_bounds__(C::THREADS)
   const int b_first = seq_at(prefix, a.B, s0);
 
   // ------------------------------------------------------------------ producer
-  if (warp == C::NG) {
+  if (warp == C::NCW) {
     if (lane != 0) return;
     int k = 0;
     bool ok = true;
+    // The cache is read once per step: mark its lines first to evict so the
+    // partials, queries and outputs of the step stay in L2.
+    const uint64_t pol = policy_evict_first();
+#define GVA_TMA(dst, map, x, y, bar) tma_load_2d_hint(dst, map, x, y, bar, pol)
     for (int b = b_first; ok && b < a.B && prefix[b] < s1; ++b) {
       const int j0 = max(s0, prefix[b]) - prefix[b], j1 = min(s1, prefix[b + 1]) - prefix[b];
-      const int row0 = __ldg(a.seq_offset + b);
+      const int row0 = offs[b];
       for (int t0 = j0; t0 < j1; t0 += C::TT, ++k) {
         const int s = k % C::STAGES;
         if (k >= C::STAGES &&
@@ -112,6 +140,7 @@ __global__ void __launch_bounds__(C::THREADS)
           break;
         }
         const uint32_t fb = smem_u32(full + s);
+        if (k == 0) trace_mark(a, 2);
         mbar_arrive_expect_tx(fb, C::TX);
         const uint32_t st = smem_u32(pipe + s * C::STAGE);
         const int y = row0 + t0;
@@ -119,18 +148,18 @@ __global__ void __launch_bounds__(C::THREADS)
         for (int g = 0; g < C::NG; ++g)
 #pragma unroll
           for (int c = 0; c < C::CB; ++c)
-            tma_load_2d(st + (g * C::CB + c) * C::BOX, &tm_x, g * C::D_H + c * 64, y, fb);
+            GVA_TMA(st + (g * C::CB + c) * C::BOX, &tm_x, g * C::D_H + c * 64, y, fb);
         if constexpr (C::GQA) {
 #pragma unroll
           for (int g = 0; g < C::NG; ++g)
 #pragma unroll
             for (int c = 0; c < C::CB; ++c)
-              tma_load_2d(st + C::XB + (g * C::CB + c) * C::BOX, &tm_v, g * C::D_H + c * 64, y,
-                          fb);
+              GVA_TMA(st + C::XB + (g * C::CB + c) * C::BOX, &tm_v, g * C::D_H + c * 64, y, fb);
         }
-        if constexpr (C::DRP > 0) tma_load_2d(st + C::XB, &tm_kr, 0, y, fb);
+        if constexpr (C::DRP > 0) GVA_TMA(st + C::XB, &tm_kr, 0, y, fb);
       }
     }
+#undef GVA_TMA
     // Drain: do not leave while a copy into this CTA's shared memory is in flight.
     for (int kk = max(0, k - C::STAGES); kk < k; ++kk)
       mbar_wait(smem_u32(full + kk % C::STAGES), (kk / C::STAGES) & 1, a.status);
@@ -138,17 +167,21 @@ __global__ void __launch_bounds__(C::THREADS)
   }
 
   // ------------------------------------------------------------------ consumers
-  const int g = warp;
+  // warp = g * W + w: group g, m-tiles w*MW .. w*MW+MW-1 of every tile
+  const int g = warp / C::W, w = warp % C::W;
   const int t = lane & 3, gq = lane >> 2;
   const int mi = lane >> 3, r8 = lane & 7;
   // ldmatrix row/chunk owned by this lane (see the fragment layouts of m16n8k16)
-  const int a_row = (mi & 1) * 8 + r8, a_kc = mi >> 1;     // scores A: rows=tokens
-  const int v_tok = (mi >> 1) * 8 + r8, v_dc = mi & 1;     // P.V A (trans): rows=tokens
+  const int a_row = w * C::MW * 16 + (mi & 1) * 8 + r8, a_kc = mi >> 1;   // scores A: rows = tokens
+  const int v_tok = w * C::MW * 16 + (mi >> 1) * 8 + r8, v_dc = mi & 1;   // P.V A (trans)
   const int H = a.H;
   const int dq = C::D_H + a.d_r;
-  // columns owned after the hi/lo merge: heads h_lo, h_lo+1 of this group
+  // columns owned after the hi/lo merge: heads hcol, hcol+1 of this group
   const int hcol = (2 * t) & (C::HPG - 1);
   const bool lo_half = (C::HPG == 4) && (t >= 2);
+  float* mg_ml = merge + g * (C::MERGE_ML + C::MERGE_O);
+  float* mg_o = mg_ml + C::MERGE_ML;
+  bool ok = true;   // false once a bounded wait gave up: skip work, keep barrier order
 
   int k = 0;
   for (int b = b_first; b < a.B && prefix[b] < s1; ++b) {
@@ -164,40 +197,43 @@ __global__ void __launch_bounds__(C::THREADS)
       const bool lo = C::HPG == 8 ? (nt == 1) : (gq >= 4);
       const int head = g * C::HPG + hl;
       float v[C::KS][4];
-      float w[C::RS > 0 ? C::RS : 1][4];
+      float wv[C::RS > 0 ? C::RS : 1][4];
       if constexpr (!C::GQA) {
         const float* qrow = a.q_abs + ((size_t)b * H + head) * dq;
 #pragma unroll
         for (int ks = 0; ks < C::KS; ++ks) {
           const int k0 = ks * 16 + 2 * t;
-          v[ks][0] = qrow[k0];
-          v[ks][1] = qrow[k0 + 1];
-          v[ks][2] = qrow[k0 + 8];
-          v[ks][3] = qrow[k0 + 9];
+          const float2 x01 = *reinterpret_cast<const float2*>(qrow + k0);
+          const float2 x89 = *reinterpret_cast<const float2*>(qrow + k0 + 8);
+          v[ks][0] = x01.x;
+          v[ks][1] = x01.y;
+          v[ks][2] = x89.x;
+          v[ks][3] = x89.y;
         }
 #pragma unroll
         for (int rs = 0; rs < C::RS; ++rs) {
           const int k0 = rs * 16 + 2 * t;
-          const int kk[4] = {k0, k0 + 1, k0 + 8, k0 + 9};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) w[rs][e] = kk[e] < a.d_r ? qrow[C::D_H + kk[e]] : 0.f;
+          wv[rs][0] = k0 < a.d_r ? qrow[C::D_H + k0] : 0.f;
+          wv[rs][1] = k0 + 1 < a.d_r ? qrow[C::D_H + k0 + 1] : 0.f;
+          wv[rs][2] = k0 + 8 < a.d_r ? qrow[C::D_H + k0 + 8] : 0.f;
+          wv[rs][3] = k0 + 9 < a.d_r ? qrow[C::D_H + k0 + 9] : 0.f;
         }
       } else {
         const size_t base = ((size_t)b * H + head) * C::D_H;
 #pragma unroll
         for (int ks = 0; ks < C::KS; ++ks) {
           const int k0 = ks * 16 + 2 * t;
-          const int kk[4] = {k0, k0 + 1, k0 + 8, k0 + 9};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            float x = a.q_bf16
-                          ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.q_raw)[base + kk[e]])
-                          : reinterpret_cast<const float*>(a.q_raw)[base + kk[e]];
+            const int kk = k0 + (e & 1) + (e >> 1) * 8;
+            const float x = a.q_bf16
+                ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.q_raw)[base + kk])
+                : reinterpret_cast<const float*>(a.q_raw)[base + kk];
             v[ks][e] = x * a.q_scale;
           }
         }
       }
-      auto part = [&](float x) { float h = bf16_round(x); return lo ? x - h : h; };
+      auto part = [&](float x) { const float h = bf16_round(x); return lo ? x - h : h; };
 #pragma unroll
       for (int ks = 0; ks < C::KS; ++ks) {
         qb[nt][ks][0] = pack_bf16(part(v[ks][0]), part(v[ks][1]));
@@ -205,8 +241,8 @@ __global__ void __launch_bounds__(C::THREADS)
       }
 #pragma unroll
       for (int rs = 0; rs < C::RS; ++rs) {
-        qr[nt][rs][0] = pack_bf16(part(w[rs][0]), part(w[rs][1]));
-        qr[nt][rs][1] = pack_bf16(part(w[rs][2]), part(w[rs][3]));
+        qr[nt][rs][0] = pack_bf16(part(wv[rs][0]), part(wv[rs][1]));
+        qr[nt][rs][1] = pack_bf16(part(wv[rs][2]), part(wv[rs][3]));
       }
     }
 
@@ -221,66 +257,75 @@ __global__ void __launch_bounds__(C::THREADS)
 
     for (int t0 = j0; t0 < j1; t0 += C::TT, ++k) {
       const int s = k % C::STAGES;
-      if (!mbar_wait(smem_u32(full + s), (k / C::STAGES) & 1, a.status)) return;
+      if (ok) ok = mbar_wait(smem_u32(full + s), (k / C::STAGES) & 1, a.status);
+      if (!ok) continue;
+      if (warp == 0 && lane == 0 && k == 0) trace_mark(a, 3);
       const int nvalid = min(C::TT, j1 - t0);
       uint8_t* st = pipe + s * C::STAGE;
       uint8_t* xg = st + g * C::CB * C::BOX;
       uint8_t* vg = C::GQA ? st + C::XB + g * C::CB * C::BOX : xg;
-      if (nvalid < C::TT) {
-        // rows past the sequence may hold anything (even NaN): zero them so
-        // that p = 0 really contributes nothing to P.V
-        const int nz = C::TT - nvalid;
+      const int r_lo = w * C::MW * 16, r_hi = r_lo + C::MW * 16;   // this warp's rows
+      const bool ragged = nvalid < r_hi;
+      if (ragged) {
+        // rows past the sequence may hold anything (even NaN): zero this warp's
+        // rows so that p = 0 really contributes nothing to P.V
+        const int r0 = max(nvalid, r_lo), nz = r_hi - r0;
         for (int e = lane; e < nz * 8 * C::CB; e += 32) {
-          const int c = e / (nz * 8), rr = nvalid + (e >> 3) % nz, ch = e & 7;
+          const int c = e / (nz * 8), rr = r0 + (e >> 3) % nz, ch = e & 7;
           *reinterpret_cast<uint4*>(vg + c * C::BOX + rr * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
         }
         __syncwarp();
       }
       const uint32_t xg_u = smem_u32(xg), vg_u = smem_u32(vg), kr_u = smem_u32(st + C::XB);
 
-      // ---- scores
-      float sc[C::MT][4];
+      // ---- scores of this warp's MW*16 tokens (two accumulator chains per m-tile)
+      float sc[C::MW][4];
 #pragma unroll
-      for (int mt = 0; mt < C::MT; ++mt) {
-        float acc[C::NT][4];
+      for (int mm = 0; mm < C::MW; ++mm) {
+        const int arow = a_row + mm * 16;
+        float acc[2][C::NT][4];
 #pragma unroll
-        for (int nt = 0; nt < C::NT; ++nt)
+        for (int c2 = 0; c2 < 2; ++c2)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-        const int row = mt * 16 + a_row;
+          for (int nt = 0; nt < C::NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[c2][nt][e] = 0.f;
 #pragma unroll
         for (int ks = 0; ks < C::KS; ++ks) {
           uint32_t a0, a1, a2, a3;
-          const uint32_t addr = xg_u + (ks >> 2) * C::BOX + row * 128 +
-                                ((((ks & 3) * 2 + a_kc) ^ r8) << 4);
-          ldsm_x4(addr, a0, a1, a2, a3);
+          ldsm_x4(xg_u + (ks >> 2) * C::BOX + arow * 128 + ((((ks & 3) * 2 + a_kc) ^ r8) << 4), a0,
+                  a1, a2, a3);
 #pragma unroll
-          for (int nt = 0; nt < C::NT; ++nt) mma_bf16(acc[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
+          for (int nt = 0; nt < C::NT; ++nt)
+            mma_bf16(acc[ks & 1][nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
         }
 #pragma unroll
         for (int rs = 0; rs < C::RS; ++rs) {
           uint32_t a0, a1, a2, a3;
-          const uint32_t addr = kr_u + swz<C::KR_SW>(row * C::DRP * 2 + (rs * 2 + a_kc) * 16);
-          ldsm_x4(addr, a0, a1, a2, a3);
+          ldsm_x4(kr_u + swz<C::KR_SW>(arow * C::DRP * 2 + (rs * 2 + a_kc) * 16), a0, a1, a2, a3);
 #pragma unroll
-          for (int nt = 0; nt < C::NT; ++nt) mma_bf16(acc[nt], a0, a1, a2, a3, qr[nt][rs][0], qr[nt][rs][1]);
+          for (int nt = 0; nt < C::NT; ++nt)
+            mma_bf16(acc[(C::KS + rs) & 1][nt], a0, a1, a2, a3, qr[nt][rs][0], qr[nt][rs][1]);
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           float x;
-          if constexpr (C::HPG == 8) x = acc[0][e] + acc[1][e];
-          else x = acc[0][e] + __shfl_xor_sync(0xffffffffu, acc[0][e], 2);
-          const int r = mt * 16 + gq + (e >= 2 ? 8 : 0);
-          sc[mt][e] = r < nvalid ? x : -INFINITY;
+          if constexpr (C::HPG == 8) x = (acc[0][0][e] + acc[1][0][e]) + (acc[0][1][e] + acc[1][1][e]);
+          else {
+            x = acc[0][0][e] + acc[1][0][e];
+            x += __shfl_xor_sync(0xffffffffu, x, 2);
+          }
+          const int r = r_lo + mm * 16 + gq + (e >= 2 ? 8 : 0);
+          sc[mm][e] = r < nvalid ? x : -INFINITY;
         }
       }
 
       // ---- online softmax (fp32, base 2); this thread owns heads hcol, hcol+1
       float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-      for (int mt = 0; mt < C::MT; ++mt) {
-        mx0 = fmaxf(mx0, fmaxf(sc[mt][0], sc[mt][2]));
-        mx1 = fmaxf(mx1, fmaxf(sc[mt][1], sc[mt][3]));
+      for (int mm = 0; mm < C::MW; ++mm) {
+        mx0 = fmaxf(mx0, fmaxf(sc[mm][0], sc[mm][2]));
+        mx1 = fmaxf(mx1, fmaxf(sc[mm][1], sc[mm][3]));
       }
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
@@ -288,26 +333,29 @@ __global__ void __launch_bounds__(C::THREADS)
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
       }
       const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
+      // a warp may see no valid token yet (its rows all past the piece end):
+      // exponentiate against 0 then, so that p = 0 and alpha = 0, never NaN
+      const float ms0 = mn0 == -INFINITY ? 0.f : mn0, ms1 = mn1 == -INFINITY ? 0.f : mn1;
+      const float al0 = ex2(m0 - ms0), al1 = ex2(m1 - ms1);
       m0 = mn0;
       m1 = mn1;
       float rs0 = 0.f, rs1 = 0.f;
-      uint32_t bp[C::NT][C::MT][2];
+      uint32_t bp[C::MW][C::NT][2];
 #pragma unroll
-      for (int mt = 0; mt < C::MT; ++mt) {
-        const float p0 = ex2(sc[mt][0] - m0), p1 = ex2(sc[mt][1] - m1);
-        const float p2 = ex2(sc[mt][2] - m0), p3 = ex2(sc[mt][3] - m1);
+      for (int mm = 0; mm < C::MW; ++mm) {
+        const float p0 = ex2(sc[mm][0] - ms0), p1 = ex2(sc[mm][1] - ms1);
+        const float p2 = ex2(sc[mm][2] - ms0), p3 = ex2(sc[mm][3] - ms1);
         rs0 += p0 + p2;
         rs1 += p1 + p3;
         const float h0 = bf16_round(p0), h1 = bf16_round(p1), h2 = bf16_round(p2), h3 = bf16_round(p3);
         if constexpr (C::HPG == 8) {
-          bp[0][mt][0] = movm_t(pack_bf16(h0, h1));
-          bp[0][mt][1] = movm_t(pack_bf16(h2, h3));
-          bp[1][mt][0] = movm_t(pack_bf16(p0 - h0, p1 - h1));
-          bp[1][mt][1] = movm_t(pack_bf16(p2 - h2, p3 - h3));
+          bp[mm][0][0] = movm_t(pack_bf16(h0, h1));
+          bp[mm][0][1] = movm_t(pack_bf16(h2, h3));
+          bp[mm][1][0] = movm_t(pack_bf16(p0 - h0, p1 - h1));
+          bp[mm][1][1] = movm_t(pack_bf16(p2 - h2, p3 - h3));
         } else {
-          bp[0][mt][0] = movm_t(lo_half ? pack_bf16(p0 - h0, p1 - h1) : pack_bf16(h0, h1));
-          bp[0][mt][1] = movm_t(lo_half ? pack_bf16(p2 - h2, p3 - h3) : pack_bf16(h2, h3));
+          bp[mm][0][0] = movm_t(lo_half ? pack_bf16(p0 - h0, p1 - h1) : pack_bf16(h0, h1));
+          bp[mm][0][1] = movm_t(lo_half ? pack_bf16(p2 - h2, p3 - h3) : pack_bf16(h2, h3));
         }
       }
       l0 = l0 * al0 + rs0;
@@ -322,32 +370,93 @@ __global__ void __launch_bounds__(C::THREADS)
           o[nt][md][3] *= al1;
         }
 
-      // ---- O^T += V^T P
+      // ---- O^T += V^T P over this warp's tokens
 #pragma unroll
-      for (int mt = 0; mt < C::MT; ++mt) {
-        const int tok = mt * 16 + v_tok;
+      for (int mm = 0; mm < C::MW; ++mm) {
+        const int vt = v_tok + mm * 16;
 #pragma unroll
         for (int md = 0; md < C::KS; ++md) {
           uint32_t a0, a1, a2, a3;
-          const uint32_t addr = vg_u + (md >> 2) * C::BOX + tok * 128 +
-                                ((((md & 3) * 2 + v_dc) ^ r8) << 4);
-          ldsm_x4_t(addr, a0, a1, a2, a3);
+          ldsm_x4_t(vg_u + (md >> 2) * C::BOX + vt * 128 + ((((md & 3) * 2 + v_dc) ^ r8) << 4), a0,
+                    a1, a2, a3);
 #pragma unroll
           for (int nt = 0; nt < C::NT; ++nt)
-            mma_bf16(o[nt][md], a0, a1, a2, a3, bp[nt][mt][0], bp[nt][mt][1]);
+            mma_bf16(o[nt][md], a0, a1, a2, a3, bp[mm][nt][0], bp[mm][nt][1]);
         }
       }
-      if (nvalid < C::TT) fence_proxy_async_smem();
+      if (ragged) fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(empty + s));
     }
 
-    // ---- piece epilogue: un-normalised partial (m, l, o) to slot blockIdx.x + b
+    // ---- piece epilogue
+    if (warp == 0 && lane == 0) trace_mark(a, 4);
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
       l0 += __shfl_xor_sync(0xffffffffu, l0, off);
       l1 += __shfl_xor_sync(0xffffffffu, l1, off);
     }
+    if constexpr (C::W > 1) {
+      // merge the W warps of this group: common max, rescale, sum through smem
+      const int bar = 1 + g, nthr = C::W * 32;
+      if (gq == 0) {
+        float* e = mg_ml + (w * 4 + t) * 4;
+        e[0] = m0; e[1] = m1; e[2] = l0; e[3] = l1;
+      }
+      named_bar_sync(bar, nthr);
+      float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < C::W; ++u) {
+        M0 = fmaxf(M0, mg_ml[(u * 4 + t) * 4 + 0]);
+        M1 = fmaxf(M1, mg_ml[(u * 4 + t) * 4 + 1]);
+      }
+      float L0 = 0.f, L1 = 0.f;
+#pragma unroll
+      for (int u = 0; u < C::W; ++u) {
+        const float* e = mg_ml + (u * 4 + t) * 4;
+        L0 += e[2] * ex2(e[0] - M0);
+        L1 += e[3] * ex2(e[1] - M1);
+      }
+      const float f0 = ex2(m0 - M0), f1 = ex2(m1 - M1);
+#pragma unroll
+      for (int nt = 0; nt < C::NT; ++nt)
+#pragma unroll
+        for (int md = 0; md < C::KS; ++md) {
+          o[nt][md][0] *= f0;
+          o[nt][md][1] *= f1;
+          o[nt][md][2] *= f0;
+          o[nt][md][3] *= f1;
+        }
+      m0 = M0; m1 = M1; l0 = L0; l1 = L1;
+      if (w > 0) {
+        float* dst = mg_o + ((w - 1) * 32 + lane) * (C::NT * C::KS * 4);
+#pragma unroll
+        for (int nt = 0; nt < C::NT; ++nt)
+#pragma unroll
+          for (int md = 0; md < C::KS; ++md)
+            *reinterpret_cast<float4*>(dst + (nt * C::KS + md) * 4) =
+                make_float4(o[nt][md][0], o[nt][md][1], o[nt][md][2], o[nt][md][3]);
+      }
+      named_bar_sync(bar, nthr);
+      if (w == 0) {
+#pragma unroll
+        for (int u = 1; u < C::W; ++u) {
+          const float* src = mg_o + ((u - 1) * 32 + lane) * (C::NT * C::KS * 4);
+#pragma unroll
+          for (int nt = 0; nt < C::NT; ++nt)
+#pragma unroll
+            for (int md = 0; md < C::KS; ++md) {
+              const float4 x = *reinterpret_cast<const float4*>(src + (nt * C::KS + md) * 4);
+              o[nt][md][0] += x.x;
+              o[nt][md][1] += x.y;
+              o[nt][md][2] += x.z;
+              o[nt][md][3] += x.w;
+            }
+        }
+      }
+      named_bar_sync(bar, nthr);   // scratch free for the next piece
+    }
+    if (w != 0) continue;
 #pragma unroll
     for (int md = 0; md < C::KS; ++md)
 #pragma unroll
@@ -355,7 +464,7 @@ __global__ void __launch_bounds__(C::THREADS)
         if constexpr (C::HPG == 8) o[0][md][e] += o[1][md][e];
         else o[0][md][e] += __shfl_xor_sync(0xffffffffu, o[0][md][e], 2);
       }
-    if (C::HPG == 8 || t < 2) {
+    if (ok && (C::HPG == 8 || t < 2)) {
       const size_t slot = (size_t)blockIdx.x + b;
       const int h0 = g * C::HPG + hcol;
       float* po0 = a.part_o + (slot * H + h0) * C::D_H;
@@ -373,6 +482,7 @@ __global__ void __launch_bounds__(C::THREADS)
         a.part_ml[slot * H + h0 + 1] = make_float2(m1, l1);
       }
     }
+    if (warp == 0 && lane == 0) trace_mark(a, 5);
   }
 }
 

@@ -67,6 +67,8 @@ __global__ void __launch_bounds__(kSimtThreads)
   const T* Vv = reinterpret_cast<const T*>(a.Vv);
   const T* KR = reinterpret_cast<const T*>(a.KR);
 
+  pdl_wait();
+  pdl_trigger();
   long long total64 = block_scan_lengths(a.seq_len, a.B, prefix, wtmp);
   int total = (int)total64;
   if (total64 >= (1ll << 31)) {
@@ -206,8 +208,7 @@ cudaError_t launch_decode_simt(const gva_shape_t& sh, bool gqa, DecodeArgs& a, c
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Ly.total);
     if (e != cudaSuccess) return e;
   }
-  k<<<a.grid, kSimtThreads, Ly.total, st>>>(a, Ly, gqa ? 1 : 0);
-  return cudaGetLastError();
+  return launch_pdl(k, dim3(a.grid), dim3(kSimtThreads), Ly.total, st, a, Ly, gqa ? 1 : 0);
 }
 
 }  // namespace gva

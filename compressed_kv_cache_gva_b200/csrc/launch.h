@@ -7,12 +7,36 @@
 
 #include "../../include/gva.h"
 
+#include <utility>
+
 namespace gva {
 
 struct DecodeArgs;
 
+// Launch with programmatic stream serialization allowed (see pdl_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  // Every kernel asks for the maximum shared-memory carveout, so consecutive
+  // kernels never force the SM to reconfigure its L1/shared split in between.
+  cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                       (int)cudaSharedmemCarveoutMaxShared);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
+}
+
 cudaError_t launch_absorb(const gva_shape_t& sh, const void* q, const void* M, const int* q_pos,
                           float* q_abs, float c, cudaStream_t st);
+size_t absorb_smem_bytes(const gva_shape_t& sh);
 
 cudaError_t launch_append(const gva_shape_t& sh, int N, const void* v_new, const void* kpe_new,
                           const int* slot, const int* pos, long long num_slots, void* V_cache,

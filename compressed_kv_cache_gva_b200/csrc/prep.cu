@@ -33,118 +33,216 @@ __device__ __forceinline__ void store_rounded<__nv_bfloat16>(__nv_bfloat16* p, d
   *p = f64_to_bf16_rne(x);
 }
 
-// Rotation of pair (i, i + d_r/2) at position pos; angle in float64.
-__device__ __forceinline__ void rope_pair(double x1, double x2, double pos, int i, int d_r,
-                                          double base, double& y1, double& y2) {
-  const double inv_freq = pow(base, -2.0 * (double)i / (double)d_r);
+// Rotation of pair (i, i + d_r/2) at position pos; the angle pos * base^(-2i/d_r)
+// is formed in float64 from a float64 frequency table.
+__device__ __forceinline__ void rope_pair(double x1, double x2, double pos, double inv_freq,
+                                          double& y1, double& y2) {
   double s, c;
   sincos(pos * inv_freq, &s, &c);
   y1 = x1 * c - x2 * s;
   y2 = x1 * s + x2 * c;
 }
 
-// One CTA per head h: M_h staged in shared memory as float, then every query of
-// the batch is multiplied by it.  Thread i < d_h owns output element i.
-template <typename TQ>
-__global__ void absorb_query_kernel(int B, int H, int d_h, int d_n, int d_r, double base,
-                                    float c, const TQ* __restrict__ q, const TQ* __restrict__ M,
-                                    const int* __restrict__ q_pos, float* __restrict__ q_abs) {
-  extern __shared__ float sm[];
-  float* Ms = sm;                       // [d_h][d_n + 1] (padded row)
-  float* qs = sm + d_h * (d_n + 1);     // [d_n + d_r]
-  const int h = blockIdx.x;
-  const int ld = d_n + 1;
-  for (int e = threadIdx.x; e < d_h * d_n; e += blockDim.x)
-    Ms[(e / d_n) * ld + (e % d_n)] = to_f32(M[(size_t)h * d_h * d_n + e]);
-  const int dq = d_n + d_r, dout = d_h + d_r;
-  for (int b = 0; b < B; ++b) {
-    __syncthreads();
-    for (int e = threadIdx.x; e < dq; e += blockDim.x)
-      qs[e] = to_f32(q[((size_t)b * H + h) * dq + e]);
-    __syncthreads();
-    float* o = q_abs + ((size_t)b * H + h) * dout;
-    for (int i = threadIdx.x; i < d_h; i += blockDim.x) {
-      float acc = 0.f;
-      const float* row = Ms + i * ld;
-      for (int k = 0; k < d_n; ++k) acc = fmaf(qs[k], row[k], acc);
-      o[i] = acc * c;
+constexpr int kAbsorbQueries = 4;   // queries per CTA
+constexpr int kAbsorbVecs = 16;     // 16-byte vectors of an M_h row held in registers
+
+// 8 bf16 (or 4 float) elements of a 16-byte vector, widened to float.
+template <typename T> struct Vec16;
+template <> struct Vec16<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void widen(const uint4& u, float* out) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      out[2 * i] = __uint_as_float(w[i] << 16);
+      out[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
     }
+  }
+};
+template <> struct Vec16<float> {
+  static constexpr int N = 4;
+  __device__ static void widen(const uint4& u, float* out) {
+    out[0] = __uint_as_float(u.x); out[1] = __uint_as_float(u.y);
+    out[2] = __uint_as_float(u.z); out[3] = __uint_as_float(u.w);
+  }
+};
+
+// grid (H, ceil(B / 4), ceil(d_h / 32)), 8 warps.  Warp w < 4 computes 32
+// elements of q~ for query b0 + w (lane = one row of M_h, whose 16-byte vectors
+// are all requested before the first FMA); warp 4 + w rotates the positional
+// slice of the same query (float64 angle; CTAs with z == 0 only).  Everything is
+// computed before waiting on the preceding kernel (it reads caller inputs only);
+// only the stores of q_abs come after.
+template <typename TQ>
+__global__ void __launch_bounds__(2 * kAbsorbQueries * 32)
+    absorb_query_kernel(int B, int H, int d_h, int d_n, int d_r, float c, const TQ* __restrict__ q,
+                        const TQ* __restrict__ M, const int* __restrict__ q_pos,
+                        float* __restrict__ q_abs, const RopeTable rt) {
+  extern __shared__ float sm[];
+  const int dq = d_n + d_r, dout = d_h + d_r;
+  const int h = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qi = warp % kAbsorbQueries;
+  const int b = blockIdx.y * kAbsorbQueries + qi;
+  float* qv = sm + qi * dq;
+  const bool active = b < B;
+  const TQ* qrow = q + ((size_t)(active ? b : 0) * H + h) * dq;
+  float* o = q_abs + ((size_t)(active ? b : 0) * H + h) * dout;
+  if (warp < kAbsorbQueries) {
+    const int i = blockIdx.z * 32 + lane;               // output element of this lane
+    const bool row_ok = active && i < d_h;
+    const TQ* row = M + ((size_t)h * d_h + (row_ok ? i : 0)) * d_n;
+    constexpr int V = Vec16<TQ>::N;
+    const bool vec = (d_n % V) == 0 && (reinterpret_cast<uintptr_t>(M) & 15) == 0;
+    if (active)
+      for (int e = lane; e < d_n; e += 32) qv[e] = to_f32(qrow[e]);
+    __syncwarp();
+    float acc0 = 0.f, acc1 = 0.f;
+    if (vec) {
+      for (int k0 = 0; k0 < d_n; k0 += kAbsorbVecs * V) {
+        uint4 raw[kAbsorbVecs];
+#pragma unroll
+        for (int u = 0; u < kAbsorbVecs; ++u)
+          if (row_ok && k0 + u * V < d_n) raw[u] = *reinterpret_cast<const uint4*>(row + k0 + u * V);
+#pragma unroll
+        for (int u = 0; u < kAbsorbVecs; ++u) {
+          if (!(row_ok && k0 + u * V < d_n)) continue;
+          float x[V];
+          Vec16<TQ>::widen(raw[u], x);
+#pragma unroll
+          for (int j = 0; j < V; j += 2) {
+            acc0 = fmaf(qv[k0 + u * V + j], x[j], acc0);
+            acc1 = fmaf(qv[k0 + u * V + j + 1], x[j + 1], acc1);
+          }
+        }
+      }
+    } else if (row_ok) {
+      for (int k = 0; k < d_n; ++k) acc0 = fmaf(qv[k], to_f32(row[k]), acc0);
+    }
+    pdl_wait();
+    pdl_trigger();
+    if (row_ok) o[i] = (acc0 + acc1) * c;
+  } else {
     const int half = d_r / 2;
-    for (int i = threadIdx.x; i < half; i += blockDim.x) {
-      double y1, y2;
-      rope_pair(qs[d_n + i], qs[d_n + half + i], (double)q_pos[b], i, d_r, base, y1, y2);
-      o[d_h + i] = (float)(y1 * (double)c);
-      o[d_h + half + i] = (float)(y2 * (double)c);
+    const bool rope = active && blockIdx.z == 0;
+    const double pos = rope ? (double)q_pos[b] : 0.0;
+    double y1[2] = {0.0, 0.0}, y2[2] = {0.0, 0.0};
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int p = lane + 32 * u;
+      if (rope && p < half)
+        rope_pair(to_f32(qrow[d_n + p]), to_f32(qrow[d_n + half + p]), pos, rt.inv_freq[p], y1[u],
+                  y2[u]);
+    }
+    pdl_wait();
+    pdl_trigger();
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int p = lane + 32 * u;
+      if (rope && p < half) {
+        o[d_h + p] = (float)(y1[u] * (double)c);
+        o[d_h + half + p] = (float)(y2[u] * (double)c);
+      }
     }
   }
 }
 
-// One warp per token: 16-byte copies of the value row, lanes 0..d_r/2-1 rotate
-// one pair each of the positional key.
+// One warp per token: the value row is loaded (16-byte vectors) and the
+// positional pairs rotated before waiting on the preceding kernel; the stores
+// into the cache come after.
 template <typename T>
-__global__ void append_cache_kernel(int N, int row_elems, int d_r, double base,
-                                    const T* __restrict__ v_new, const T* __restrict__ kpe_new,
-                                    const int* __restrict__ slot, const int* __restrict__ pos,
-                                    long long num_slots, T* __restrict__ V_cache,
-                                    T* __restrict__ kr_cache, int* __restrict__ err_flag) {
+__global__ void append_cache_kernel(int N, int row_elems, int d_r, const T* __restrict__ v_new,
+                                    const T* __restrict__ kpe_new, const int* __restrict__ slot,
+                                    const int* __restrict__ pos, long long num_slots,
+                                    T* __restrict__ V_cache, T* __restrict__ kr_cache,
+                                    int* __restrict__ err_flag, const RopeTable rt) {
+  constexpr int kVecPerLane = 4;   // rows up to 32*4*16 bytes = 2 KB in registers
   const int warps = blockDim.x >> 5;
   const int lane = threadIdx.x & 31;
-  for (long long i = (long long)blockIdx.x * warps + (threadIdx.x >> 5); i < N;
-       i += (long long)gridDim.x * warps) {
-    const long long s = slot[i];
-    if (s < 0 || s >= num_slots) {
-      if (lane == 0 && err_flag) atomicExch(err_flag, 1);
-      continue;
-    }
-    const int vec = 16 / sizeof(T);
-    const uint4* src = reinterpret_cast<const uint4*>(v_new + i * row_elems);
-    uint4* dst = reinterpret_cast<uint4*>(V_cache + s * row_elems);
-    for (int e = lane; e < row_elems / vec; e += 32) dst[e] = src[e];
-    const int half = d_r / 2;
-    for (int p = lane; p < half; p += 32) {
-      double y1, y2;
+  const long long i = (long long)blockIdx.x * warps + (threadIdx.x >> 5);
+  const bool active = i < N;
+  const long long s = active ? slot[i] : -1;
+  const bool ok = active && s >= 0 && s < num_slots;
+  const int vec = 16 / sizeof(T);
+  const int nvec = row_elems / vec;
+  const uint4* src = reinterpret_cast<const uint4*>(v_new + (ok ? i : 0) * row_elems);
+  uint4 r[kVecPerLane];
+#pragma unroll
+  for (int u = 0; u < kVecPerLane; ++u)
+    if (ok && lane + 32 * u < nvec) r[u] = src[lane + 32 * u];
+  const int half = d_r / 2;
+  double y1[2] = {0.0, 0.0}, y2[2] = {0.0, 0.0};   // d_r <= 128: two pairs per lane at most
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int p = lane + 32 * u;
+    if (ok && p < half)
       rope_pair((double)to_f32(kpe_new[i * d_r + p]), (double)to_f32(kpe_new[i * d_r + half + p]),
-                (double)pos[i], p, d_r, base, y1, y2);
-      store_rounded(kr_cache + s * d_r + p, y1);
-      store_rounded(kr_cache + s * d_r + half + p, y2);
+                (double)pos[i], rt.inv_freq[p], y1[u], y2[u]);
+  }
+  pdl_wait();
+  pdl_trigger();
+  if (active && !ok) {
+    if (lane == 0 && err_flag) atomicExch(err_flag, 1);
+    return;
+  }
+  if (!ok) return;
+  uint4* dst = reinterpret_cast<uint4*>(V_cache + s * row_elems);
+#pragma unroll
+  for (int u = 0; u < kVecPerLane; ++u)
+    if (lane + 32 * u < nvec) dst[lane + 32 * u] = r[u];
+  for (int e = lane + 32 * kVecPerLane; e < nvec; e += 32) dst[e] = src[e];   // wider rows
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int p = lane + 32 * u;
+    if (p < half) {
+      store_rounded(kr_cache + s * d_r + p, y1[u]);
+      store_rounded(kr_cache + s * d_r + half + p, y2[u]);
     }
   }
+}
+
+static RopeTable rope_table(const gva_shape_t& sh) {
+  RopeTable t{};
+  for (int i = 0; i < sh.d_r / 2 && i < kMaxRopePairs; ++i)
+    t.inv_freq[i] = pow(sh.rope_base, -2.0 * (double)i / (double)sh.d_r);
+  return t;
+}
+
+size_t absorb_smem_bytes(const gva_shape_t& sh) {
+  return sizeof(float) * (size_t)kAbsorbQueries * (sh.d_n + sh.d_r);
 }
 
 cudaError_t launch_absorb(const gva_shape_t& sh, const void* q, const void* M, const int* q_pos,
                           float* q_abs, float c, cudaStream_t st) {
-  const size_t smem = sizeof(float) * ((size_t)sh.d_h * (sh.d_n + 1) + sh.d_n + sh.d_r);
-  const int threads = 128;
+  const size_t smem = absorb_smem_bytes(sh);
+  const dim3 grid(sh.H, (sh.B + kAbsorbQueries - 1) / kAbsorbQueries, (sh.d_h + 31) / 32);
+  const dim3 block(2 * kAbsorbQueries * 32);
+  const RopeTable rt = rope_table(sh);
   if (sh.q_dtype == GVA_BF16) {
     auto k = absorb_query_kernel<__nv_bfloat16>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<sh.H, threads, smem, st>>>(sh.B, sh.H, sh.d_h, sh.d_n, sh.d_r, sh.rope_base, c,
-                                   (const __nv_bfloat16*)q, (const __nv_bfloat16*)M, q_pos, q_abs);
-  } else {
-    auto k = absorb_query_kernel<float>;
-    if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<sh.H, threads, smem, st>>>(sh.B, sh.H, sh.d_h, sh.d_n, sh.d_r, sh.rope_base, c,
-                                   (const float*)q, (const float*)M, q_pos, q_abs);
+    return launch_pdl(k, grid, block, smem, st, sh.B, sh.H, sh.d_h, sh.d_n, sh.d_r, c,
+                      (const __nv_bfloat16*)q, (const __nv_bfloat16*)M, q_pos, q_abs, rt);
   }
-  return cudaGetLastError();
+  auto k = absorb_query_kernel<float>;
+  if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  return launch_pdl(k, grid, block, smem, st, sh.B, sh.H, sh.d_h, sh.d_n, sh.d_r, c, (const float*)q,
+                    (const float*)M, q_pos, q_abs, rt);
 }
 
 cudaError_t launch_append(const gva_shape_t& sh, int N, const void* v_new, const void* kpe_new,
                           const int* slot, const int* pos, long long num_slots, void* V_cache,
                           void* kr_cache, int* err_flag, cudaStream_t st) {
   const int threads = 256, warps = threads / 32;
-  long long blocks = ((long long)N + warps - 1) / warps;
-  int grid = (int)(blocks < 65535 * 8 ? blocks : 65535 * 8);
+  const int grid = (int)(((long long)N + warps - 1) / warps);   // N < 2^31: fits the x grid
   const int row = sh.G * sh.d_h;
+  const RopeTable rt = rope_table(sh);
   if (sh.cache_dtype == GVA_BF16)
-    append_cache_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(
-        N, row, sh.d_r, sh.rope_base, (const __nv_bfloat16*)v_new, (const __nv_bfloat16*)kpe_new,
-        slot, pos, num_slots, (__nv_bfloat16*)V_cache, (__nv_bfloat16*)kr_cache, err_flag);
-  else
-    append_cache_kernel<float><<<grid, threads, 0, st>>>(
-        N, row, sh.d_r, sh.rope_base, (const float*)v_new, (const float*)kpe_new, slot, pos,
-        num_slots, (float*)V_cache, (float*)kr_cache, err_flag);
-  return cudaGetLastError();
+    return launch_pdl(append_cache_kernel<__nv_bfloat16>, dim3(grid), dim3(threads), 0, st, N, row,
+                      sh.d_r, (const __nv_bfloat16*)v_new, (const __nv_bfloat16*)kpe_new, slot, pos,
+                      num_slots, (__nv_bfloat16*)V_cache, (__nv_bfloat16*)kr_cache, err_flag, rt);
+  return launch_pdl(append_cache_kernel<float>, dim3(grid), dim3(threads), 0, st, N, row, sh.d_r,
+                    (const float*)v_new, (const float*)kpe_new, slot, pos, num_slots,
+                    (float*)V_cache, (float*)kr_cache, err_flag, rt);
 }
 
 }  // namespace gva
