@@ -218,6 +218,11 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
 
 }  // namespace
 
+namespace gva {
+// Lets other translation units of the library record a reason for gva_last_error.
+void set_error_message(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+}  // namespace gva
+
 extern "C" {
 
 const char* gva_status_string(gva_status_t s) {

@@ -84,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.gva_decode_attention.argtypes = [SP, P, P, P, P, P, I64, I64, P, P, P, SZ, P]
         L.gqa_decode_attention.restype = ctypes.c_int
         L.gqa_decode_attention.argtypes = [SP, P, P, P, P, P, I64, I64, P, P, P, SZ, P]
+        L.gva_decode_attention_noalloc.restype = ctypes.c_int
+        L.gva_decode_attention_noalloc.argtypes = [SP, P, P, P, P, P, I64, I64, P, P, P]
         _lib = L
     return _lib
 
@@ -155,5 +157,19 @@ def gqa_decode_attention(shape: Shape, q, K_cache, V_cache, seq_offset, seq_len,
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def decode_attention_noalloc(shape: Shape, q_abs, V_cache, kr_cache, seq_offset, seq_len,
+                             max_total_tokens: int, out, lse=None, stream=None):
+    """gva_decode_attention_noalloc: the decode for callers that cannot allocate
+    device memory; its scratch is a fixed array inside the library."""
+    _check(lib().gva_decode_attention_noalloc(
+        ctypes.byref(shape), _ptr(q_abs), _ptr(V_cache), _ptr(kr_cache), _ptr(seq_offset),
+        _ptr(seq_len), int(max_total_tokens), V_cache.shape[0], _ptr(out), _ptr(lse),
+        _stream(stream)))
+
+
 EXPORTS = ["gva_status_string", "gva_last_error", "gva_absorb_query", "gva_append_cache",
-           "gva_decode_workspace_size", "gva_decode_attention", "gqa_decode_attention"]
+           "gva_decode_workspace_size", "gva_decode_attention", "gqa_decode_attention",
+           "gva_decode_attention_noalloc"]

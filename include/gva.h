@@ -176,6 +176,41 @@ gva_status_t gqa_decode_attention(const gva_shape_t* shape, const void* q, const
                                   int64_t num_slots, void* out, float* lse, void* workspace,
                                   size_t ws_bytes, void* stream);
 
+/*
+ * gva_decode_attention_noalloc — gva_decode_attention for callers that cannot
+ * allocate device memory.  The paper has no counterpart: this is an interface
+ * convenience of this library.
+ *
+ * Some callers have no way to obtain scratch memory: code that runs while a
+ * stream is being captured into a CUDA graph (cudaMalloc is not allowed there),
+ * plug-ins that only receive input and output buffers from a host framework whose
+ * caching allocator owns all other device memory, and latency-critical paths that
+ * must not call cudaMalloc because it can synchronise the device.  This entry
+ * point needs no workspace: the split-KV scratch is a fixed array of
+ * GVA_NOALLOC_SCRATCH_BYTES in this library's own device memory, which every GPU
+ * that loads the library holds until the process exits.  It allocates nothing
+ * (no cudaMalloc, cudaFree or allocating library routine); the caller still
+ * passes every input and output, as for gva_decode_attention.
+ *
+ *   Arguments, layouts, alignment and results: as gva_decode_attention.
+ *   Errors: GVA_ERR_WORKSPACE if the shape needs more scratch than
+ *   GVA_NOALLOC_SCRATCH_BYTES (gva_decode_workspace_size tells); GVA_ERR_CUDA if
+ *   the scratch's device address cannot be found.
+ *   The first call on each device looks up the scratch's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call before
+ *   any stream capture.  Every call clears the scratch's status word on `stream`.
+ *   All calls on a device share the one scratch array, which keeps the last call's
+ *   contents: calls whose executions overlap on the GPU (different streams, or
+ *   concurrent graphs) race and give wrong results.  Serialise them.
+ */
+#define GVA_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+gva_status_t gva_decode_attention_noalloc(const gva_shape_t* shape, const float* q_abs,
+                                          const void* V_cache, const void* kr_cache,
+                                          const int32_t* seq_offset, const int32_t* seq_len,
+                                          int64_t max_total_tokens, int64_t num_slots, void* out,
+                                          float* lse, void* stream);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif
