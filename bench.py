@@ -218,8 +218,12 @@ def run_ours(args, rank, world, local):
     ws = gva.new_workspace(sh, max_total, device=dev)
 
     def step(c):
-        gva.absorb_query(sh, q, M, qpos, q_abs)
+        gva.decode_step(sh, q, M, qpos, v_new, kpe_new, slot, pos, Vs[c], KRs[c], soff, slen_step,
+                        max_total, q_abs, out, None, None, ws)
+
+    def step_separate(c):
         gva.append_cache(sh, v_new, kpe_new, slot, pos, Vs[c], KRs[c])
+        gva.absorb_query(sh, q, M, qpos, q_abs)
         gva.decode_attention(sh, q_abs, Vs[c], KRs[c], soff, slen_step, max_total, out, None, ws)
 
     def decode_only(c):
@@ -297,6 +301,12 @@ def run_ours(args, rank, world, local):
     sampler.stop()
     assert gva.workspace_status(ws) == 0, "device status word set"
 
+    # the same step as three separate calls (no early cache streaming), for reference
+    g_sep = graphs_for(step_separate, K)
+    replay(g_sep)
+    ms_sep, _, _ = timed(g_sep, K)
+    del g_sep
+
     # decode-only timing (roofline of the dominant kernel) and the GQA comparison
     g_dec = graphs_for(decode_only, K)
     replay(g_dec)
@@ -350,9 +360,8 @@ def run_ours(args, rank, world, local):
 
     def e2e_step(c):
         d_stage.copy_(h_stage, non_blocking=True)
-        gva.absorb_query(sh, eq, M, qpos, q_abs)
-        gva.append_cache(sh, ev, ek, es, ep, Vs[c], KRs[c])
-        gva.decode_attention(sh, q_abs, Vs[c], KRs[c], soff, slen_step, max_total, out, None, ws)
+        gva.decode_step(sh, eq, M, qpos, ev, ek, es, ep, Vs[c], KRs[c], soff, slen_step, max_total,
+                        q_abs, out, None, None, ws)
         h_out.copy_(out, non_blocking=True)
 
     g_e2e = graphs_for(e2e_step, K)
@@ -376,9 +385,11 @@ def run_ours(args, rank, world, local):
                    "l2": f"inputs larger than L2: {R} rotating cache copies, "
                          f"{R * cache_bytes / 2**20:.0f} MiB",
                    "parallelism": f"weak: {world} independent batch(es), one per GPU",
-                   "step": "absorb + append + decode (split + combine)", "graphs": "CUDA graphs",
+                   "step": "gva_decode_step: append + absorb + decode (split + combine)",
+                   "graphs": "CUDA graphs",
                    "decode_path": "fma" if args.fma else "tensor"},
         "steps_per_s": round(world * K / (ms * 1e-3), 1),
+        "ms_per_step_separate_calls": round(ms_sep / K, 6),
         "pct_hbm_peak": {"of_measured": round(value / world / hbm_peak, 4),
                          "of_nominal_8TBs": round(value / world / NOMINAL_HBM_GBS, 4)},
         "gqa_comparison": {

@@ -134,7 +134,9 @@ gva_status_t plan_decode(const gva_shape_t& sh, bool gqa, long long max_total, P
 gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, const void* X,
                            const void* Vv, const void* KR, const int32_t* seq_offset,
                            const int32_t* seq_len, int64_t max_total_tokens, int64_t num_slots,
-                           void* out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
+                           void* out, float* lse, void* workspace, size_t ws_bytes, void* stream,
+                           bool prefetch = false, const int32_t* new_slots = nullptr,
+                           int n_new = 0) {
   gva_status_t s = check_shape(shp, gqa);
   if (s != GVA_OK) return s;
   const gva_shape_t& sh = *shp;
@@ -180,6 +182,9 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
   a.part_ml = reinterpret_cast<float2*>(ws + p.ws.ml_off);
   a.part_o = reinterpret_cast<float*>(ws + p.ws.o_off);
   a.grid = p.grid;
+  a.prefetch = prefetch ? 1 : 0;
+  a.new_slots = new_slots;
+  a.n_new = new_slots ? n_new : 0;
 #ifdef GVA_TRACE
   a.trace = g_trace;
 #endif
@@ -244,8 +249,8 @@ const char* gva_last_error(void) { return g_err; }
 void gva_trace_set_buffer(void* dev_buf) { g_trace = static_cast<unsigned long long*>(dev_buf); }
 #endif
 
-gva_status_t gva_absorb_query(const gva_shape_t* shp, const void* q, const void* M,
-                              const int32_t* q_pos, float* q_abs, void* stream) {
+static gva_status_t absorb_impl(const gva_shape_t* shp, const void* q, const void* M,
+                                const int32_t* q_pos, float* q_abs, void* stream, bool early) {
   gva_status_t s = check_shape(shp, false);
   if (s != GVA_OK) return s;
   const gva_shape_t& sh = *shp;
@@ -257,14 +262,15 @@ gva_status_t gva_absorb_query(const gva_shape_t* shp, const void* q, const void*
   const size_t smem = gva::absorb_smem_bytes(sh);
   if (smem > 200 * 1024) return fail(GVA_ERR_UNSUPPORTED, "M_h too large for one CTA (%zu bytes)", smem);
   const float c = scale_of(sh, false) * gva::kLog2e;
-  cudaError_t e = gva::launch_absorb(sh, q, M, q_pos, q_abs, c, static_cast<cudaStream_t>(stream));
+  cudaError_t e =
+      gva::launch_absorb(sh, q, M, q_pos, q_abs, c, static_cast<cudaStream_t>(stream), early);
   return e == cudaSuccess ? GVA_OK : cuda_fail(e, "absorb launch");
 }
 
-gva_status_t gva_append_cache(const gva_shape_t* shp, int32_t N, const void* v_new,
-                              const void* kpe_new, const int32_t* slot, const int32_t* pos,
-                              int64_t num_slots, void* V_cache, void* kr_cache, int32_t* err_flag,
-                              void* stream) {
+static gva_status_t append_impl(const gva_shape_t* shp, int32_t N, const void* v_new,
+                                const void* kpe_new, const int32_t* slot, const int32_t* pos,
+                                int64_t num_slots, void* V_cache, void* kr_cache,
+                                int32_t* err_flag, void* stream, bool early) {
   gva_status_t s = check_shape(shp, false);
   if (s != GVA_OK) return s;
   const gva_shape_t& sh = *shp;
@@ -279,8 +285,21 @@ gva_status_t gva_append_cache(const gva_shape_t* shp, int32_t N, const void* v_n
     return fail(GVA_ERR_INVALID_ARG, "value rows must be multiples of 16 bytes");
   if (num_slots < 1) return fail(GVA_ERR_INVALID_ARG, "num_slots=%lld < 1", (long long)num_slots);
   cudaError_t e = gva::launch_append(sh, N, v_new, kpe_new, slot, pos, num_slots, V_cache, kr_cache,
-                                     err_flag, static_cast<cudaStream_t>(stream));
+                                     err_flag, static_cast<cudaStream_t>(stream), early);
   return e == cudaSuccess ? GVA_OK : cuda_fail(e, "append launch");
+}
+
+gva_status_t gva_absorb_query(const gva_shape_t* shp, const void* q, const void* M,
+                              const int32_t* q_pos, float* q_abs, void* stream) {
+  return absorb_impl(shp, q, M, q_pos, q_abs, stream, false);
+}
+
+gva_status_t gva_append_cache(const gva_shape_t* shp, int32_t N, const void* v_new,
+                              const void* kpe_new, const int32_t* slot, const int32_t* pos,
+                              int64_t num_slots, void* V_cache, void* kr_cache, int32_t* err_flag,
+                              void* stream) {
+  return append_impl(shp, N, v_new, kpe_new, slot, pos, num_slots, V_cache, kr_cache, err_flag,
+                     stream, false);
 }
 
 size_t gva_decode_workspace_size(const gva_shape_t* shp, int64_t max_total_tokens) {
@@ -303,6 +322,39 @@ gva_status_t gva_decode_attention(const gva_shape_t* shape, const float* q_abs, 
                                   void* stream) {
   return decode_common(shape, false, q_abs, V_cache, V_cache, kr_cache, seq_offset, seq_len,
                        max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream);
+}
+
+gva_status_t gva_decode_step(const gva_shape_t* shape, const void* q, const void* M,
+                             const int32_t* q_pos, int32_t n_new, const void* v_new,
+                             const void* kpe_new, const int32_t* slot, const int32_t* pos,
+                             void* V_cache, void* kr_cache, int64_t num_slots,
+                             const int32_t* seq_offset, const int32_t* seq_len,
+                             int64_t max_total_tokens, float* q_abs, void* out, float* lse,
+                             int32_t* err_flag, void* workspace, size_t ws_bytes, void* stream) {
+  gva_status_t s = check_shape(shape, false);
+  if (s != GVA_OK) return s;
+  if (shape->B == 0 && n_new == 0) return GVA_OK;
+  // Validate the decode first (it has the strictest requirements), without launching.
+  if (!q_abs || !V_cache || !seq_offset || !seq_len || !out || !workspace)
+    return fail(GVA_ERR_INVALID_ARG, "a required pointer is NULL");
+  Plan p;
+  if ((s = plan_decode(*shape, false, max_total_tokens, &p)) != GVA_OK) return s;
+  if (ws_bytes < p.ws.total)
+    return fail(GVA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, p.ws.total);
+  // 1. new tokens into the cache, 2. absorbed queries, 3. decode.  This order lets
+  // the decode's split kernel start streaming the cache before it waits on the
+  // absorb kernel: absorb only triggers its successor after the append finished.
+  // Append and absorb let their successor launch immediately; every kernel still
+  // waits on its predecessor before its first store, so the chain stays ordered,
+  // and the split kernel streams all cache tiles without a new slot before it
+  // waits (its wait covers the absorb, which waited on the append).
+  if ((s = append_impl(shape, n_new, v_new, kpe_new, slot, pos, num_slots, V_cache, kr_cache,
+                       err_flag, stream, true)) != GVA_OK)
+    return s;
+  if ((s = absorb_impl(shape, q, M, q_pos, q_abs, stream, true)) != GVA_OK) return s;
+  return decode_common(shape, false, q_abs, V_cache, V_cache, kr_cache, seq_offset, seq_len,
+                       max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream,
+                       /*prefetch=*/true, slot, n_new);
 }
 
 gva_status_t gqa_decode_attention(const gva_shape_t* shape, const void* q, const void* K_cache,

@@ -58,6 +58,9 @@ struct DecodeArgs {
   float* part_o;             // [P][H][d_h] un-normalised output
   int grid;                  // CTAs of the split kernel
   int tile;                  // span granularity in tokens
+  int prefetch;              // stream the cache before the PDL wait (fused step only), except
+  const int* new_slots;      //   tiles holding one of these n_new slots, written by the
+  int n_new;                 //   append of the same step
   unsigned long long* trace; // per-CTA timestamps, only with -DGVA_TRACE (else unused)
 };
 
@@ -147,6 +150,27 @@ __device__ inline int seq_at(const int* prefix, int B, int pos) {
   }
   return lo;
 }
+
+// Walks the tiles of one CTA's span: sequence b, tile start t0 (token index in the
+// sequence) and the piece end j1.  Empty sequences are skipped; b == B means done.
+struct TileCursor {
+  int b, t0, j1;
+  __device__ void seek(const int* prefix, int B, int s0, int s1, int from) {
+    for (b = from; b < B && prefix[b] < s1; ++b) {
+      const int j0 = max(s0, prefix[b]) - prefix[b];
+      j1 = min(s1, prefix[b + 1]) - prefix[b];
+      if (j1 > j0) {
+        t0 = j0;
+        return;
+      }
+    }
+    b = B;
+  }
+  __device__ void next(const int* prefix, int B, int s0, int s1, int tile) {
+    t0 += tile;
+    if (t0 >= j1) seek(prefix, B, s0, s1, b + 1);
+  }
+};
 
 // CTA 0 records, for every sequence, where its pieces land and how many there are,
 // and flags sequences whose slots leave the cache.
@@ -305,16 +329,20 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "r"(addr));
 }
 
+// Register-only operations (movmatrix, mma) are not `volatile`: the compiler may
+// schedule them by their data dependencies, overlapping independent chains.
+// Shared-memory loads (ldmatrix) stay volatile so that they keep their place
+// after the barrier waits and the writes that produce their data.
 __device__ __forceinline__ uint32_t movm_t(uint32_t x) {
   uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
   return y;
 }
 
 // D += A * B, m16n8k16, bf16 inputs, fp32 accumulate.
 __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7},"
       " {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])

@@ -24,7 +24,7 @@
 
 namespace gva {
 
-template <int D_H_, int NG_, int HPG_, int DRP_, bool GQA_, int W_ = 1>
+template <int D_H_, int NG_, int HPG_, int DRP_, bool GQA_, int W_ = 0>
 struct MmaCfg {
   static constexpr int D_H = D_H_, NG = NG_, HPG = HPG_, DRP = GQA_ ? 0 : DRP_;
   static constexpr bool GQA = GQA_;
@@ -43,13 +43,22 @@ struct MmaCfg {
 #ifndef GVA_PIPE_BYTES   // shared memory of the stage ring per CTA (tuning knob)
 #define GVA_PIPE_BYTES (96 * 1024)
 #endif
+  // consumer warps per group (round robin over tiles).  Measured on B200: one warp
+  // per group is fastest for every workload here (a second warp per group adds the
+  // end-of-piece merge and contends for the same SM resources), so 0 means 1.
+  static constexpr int W = W_ > 0 ? W_ : 1;
   static constexpr int STAGES_RAW = GVA_PIPE_BYTES / STAGE;
-  static constexpr int STAGES = STAGES_RAW < 2 ? 2 : (STAGES_RAW > 12 ? 12 : STAGES_RAW);
+  static constexpr int STAGES_CLAMPED = STAGES_RAW < 2 ? 2 : (STAGES_RAW > 12 ? 12 : STAGES_RAW);
+  // A multiple of W: tile k lives in stage k % STAGES and is consumed by warp
+  // k % W of each group, so every stage always belongs to the same warp and that
+  // warp meets the stage's barrier phases one after another.  (With an odd stage
+  // count a warp could wait for phase p+2 while the stage is still in phase p+1,
+  // and the parity test would pass on stale data.)
+  static constexpr int STAGES = STAGES_CLAMPED / W * W < W ? W : STAGES_CLAMPED / W * W;
   static constexpr int PIPE = STAGES * STAGE;
   static constexpr uint32_t TX = XB + VB + KRB;       // bytes TMA delivers per stage
   static constexpr int MT = TT / 16;                  // 16-token m-tiles per tile
-  static constexpr int W = W_ < MT ? W_ : MT;         // consumer warps per group
-  static constexpr int MW = MT / W;                   // m-tiles per consumer warp
+  static constexpr int MW = MT;                       // m-tiles per consumer warp and tile
   static constexpr int NCW = NG * W;                  // consumer warps
   static constexpr int THREADS = (NCW + 1) * 32;
   static constexpr int NT = HPG == 8 ? 2 : 1;         // 8-column MMA tiles
@@ -62,6 +71,7 @@ struct MmaCfg {
   static constexpr int MERGE = W > 1 ? NG * (MERGE_ML + MERGE_O) * 4 : 0;  // bytes
   static constexpr int KR_SW = DRP * 2;               // swizzle span of the k_rope box
   static_assert(HPG == 4 || HPG == 8, "heads per group");
+  static_assert(STAGES % W == 0, "each stage must belong to one warp of a group");
   static_assert(D_H % 64 == 0, "d_h");
   static_assert(DRP == 0 || DRP == 16 || DRP == 32, "padded d_r");
 
@@ -92,7 +102,7 @@ __global__ void __launch_bounds__(C::THREADS, 2)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(smem_u32(full + s), 1);
-      mbar_init(smem_u32(empty + s), C::NCW);
+      mbar_init(smem_u32(empty + s), C::NG);   // one warp per group consumes a tile
     }
     fence_barrier_init();
   }
@@ -111,55 +121,97 @@ __global__ void __launch_bounds__(C::THREADS, 2)
     total = 0;
   }
   const Span sp = make_span(total, gridDim.x, C::TT);
+  const int s0 = blockIdx.x * sp.span;
+  const bool has_work = s0 < total;
+  const int s1 = min(s0 + sp.span, total);
+  const int b_first = has_work ? seq_at(prefix, a.B, s0) : a.B;
+
+  // ------------------------------------------------------------------ producer
+  // One thread issues every load of the CTA.  The cache is read once per step:
+  // its lines are marked first to evict so the partials, queries and outputs of
+  // the step stay in L2.
+  const bool producer = warp == C::NCW && lane == 0 && has_work;
+  int k_issued = 0;
+  bool prod_ok = true;
+  TileCursor cur;
+  uint64_t pol = 0;
+  auto issue = [&](int k) {
+    const int s = k % C::STAGES;
+    const uint32_t fb = smem_u32(full + s);
+    if (k == 0) trace_mark(a, 2);
+    mbar_arrive_expect_tx(fb, C::TX);
+    const uint32_t st = smem_u32(pipe + s * C::STAGE);
+    const int y = offs[cur.b] + cur.t0;
+#pragma unroll
+    for (int g = 0; g < C::NG; ++g)
+#pragma unroll
+      for (int c = 0; c < C::CB; ++c)
+        tma_load_2d_hint(st + (g * C::CB + c) * C::BOX, &tm_x, g * C::D_H + c * 64, y, fb, pol);
+    if constexpr (C::GQA) {
+#pragma unroll
+      for (int g = 0; g < C::NG; ++g)
+#pragma unroll
+        for (int c = 0; c < C::CB; ++c)
+          tma_load_2d_hint(st + C::XB + (g * C::CB + c) * C::BOX, &tm_v, g * C::D_H + c * 64, y, fb,
+                           pol);
+    }
+    if constexpr (C::DRP > 0) tma_load_2d_hint(st + C::XB, &tm_kr, 0, y, fb, pol);
+  };
+  // Fused step only: every cache row except the ones this step appends is final
+  // before this kernel launches, so the first stages are requested before the
+  // PDL wait, up to the first tile of this CTA that uses an appended row.  All
+  // threads map the appended slots onto this CTA's tile ordinals in parallel.
+  // (Rows a tile reads past its piece's end are never used, so only rows inside
+  // the pieces count.)
+  __shared__ int first_dirty;
+  if (a.prefetch) {
+    if (threadIdx.x == 0) first_dirty = 0x7fffffff;
+    __syncthreads();
+    if (has_work)
+      for (int i = threadIdx.x; i < a.n_new; i += blockDim.x) {
+        const long long sl = __ldg(a.new_slots + i);
+        int kbase = 0;
+        for (int b = b_first; b < a.B && prefix[b] < s1; ++b) {
+          const int j0 = max(s0, prefix[b]) - prefix[b], j1 = min(s1, prefix[b + 1]) - prefix[b];
+          if (j1 <= j0) continue;
+          const long long r0 = (long long)offs[b] + j0, r1 = (long long)offs[b] + j1;
+          if (sl >= r0 && sl < r1) atomicMin(&first_dirty, kbase + (int)((sl - r0) / C::TT));
+          kbase += (j1 - j0 + C::TT - 1) / C::TT;
+        }
+      }
+    __syncthreads();
+  }
+  if (producer) {
+    pol = policy_evict_first();
+    cur.seek(prefix, a.B, s0, s1, b_first);
+    if (a.prefetch) {
+      const int limit = min(C::STAGES, first_dirty);
+      for (; cur.b < a.B && k_issued < limit; ++k_issued) {
+        issue(k_issued);
+        cur.next(prefix, a.B, s0, s1, C::TT);
+      }
+    }
+  }
   pdl_wait();
   pdl_trigger();
   if (threadIdx.x == 0) trace_mark(a, 1);
   if (blockIdx.x == 0) write_meta(a, prefix, sp);
-  const int s0 = blockIdx.x * sp.span;
-  if (s0 >= total) return;
-  const int s1 = min(s0 + sp.span, total);
-  const int b_first = seq_at(prefix, a.B, s0);
+  if (!has_work) return;
 
-  // ------------------------------------------------------------------ producer
   if (warp == C::NCW) {
     if (lane != 0) return;
-    int k = 0;
-    bool ok = true;
-    // The cache is read once per step: mark its lines first to evict so the
-    // partials, queries and outputs of the step stay in L2.
-    const uint64_t pol = policy_evict_first();
-#define GVA_TMA(dst, map, x, y, bar) tma_load_2d_hint(dst, map, x, y, bar, pol)
-    for (int b = b_first; ok && b < a.B && prefix[b] < s1; ++b) {
-      const int j0 = max(s0, prefix[b]) - prefix[b], j1 = min(s1, prefix[b + 1]) - prefix[b];
-      const int row0 = offs[b];
-      for (int t0 = j0; t0 < j1; t0 += C::TT, ++k) {
-        const int s = k % C::STAGES;
-        if (k >= C::STAGES &&
-            !mbar_wait(smem_u32(empty + s), ((k / C::STAGES) - 1) & 1, a.status)) {
-          ok = false;
-          break;
-        }
-        const uint32_t fb = smem_u32(full + s);
-        if (k == 0) trace_mark(a, 2);
-        mbar_arrive_expect_tx(fb, C::TX);
-        const uint32_t st = smem_u32(pipe + s * C::STAGE);
-        const int y = row0 + t0;
-#pragma unroll
-        for (int g = 0; g < C::NG; ++g)
-#pragma unroll
-          for (int c = 0; c < C::CB; ++c)
-            GVA_TMA(st + (g * C::CB + c) * C::BOX, &tm_x, g * C::D_H + c * 64, y, fb);
-        if constexpr (C::GQA) {
-#pragma unroll
-          for (int g = 0; g < C::NG; ++g)
-#pragma unroll
-            for (int c = 0; c < C::CB; ++c)
-              GVA_TMA(st + C::XB + (g * C::CB + c) * C::BOX, &tm_v, g * C::D_H + c * 64, y, fb);
-        }
-        if constexpr (C::DRP > 0) GVA_TMA(st + C::XB, &tm_kr, 0, y, fb);
+    int k = k_issued;
+    for (; cur.b < a.B; ++k) {
+      const int s = k % C::STAGES;
+      if (k >= C::STAGES &&
+          !mbar_wait(smem_u32(empty + s), ((k / C::STAGES) - 1) & 1, a.status)) {
+        prod_ok = false;
+        break;
       }
+      issue(k);
+      cur.next(prefix, a.B, s0, s1, C::TT);
     }
-#undef GVA_TMA
+    (void)prod_ok;
     // Drain: do not leave while a copy into this CTA's shared memory is in flight.
     for (int kk = max(0, k - C::STAGES); kk < k; ++kk)
       mbar_wait(smem_u32(full + kk % C::STAGES), (kk / C::STAGES) & 1, a.status);
@@ -167,13 +219,15 @@ __global__ void __launch_bounds__(C::THREADS, 2)
   }
 
   // ------------------------------------------------------------------ consumers
-  // warp = g * W + w: group g, m-tiles w*MW .. w*MW+MW-1 of every tile
+  // warp = g * W + w: group g, tiles w, w+W, w+2W, ... of this CTA (round robin,
+  // so W tiles per group are in flight); the W running states are merged at the
+  // end of every piece
   const int g = warp / C::W, w = warp % C::W;
   const int t = lane & 3, gq = lane >> 2;
   const int mi = lane >> 3, r8 = lane & 7;
   // ldmatrix row/chunk owned by this lane (see the fragment layouts of m16n8k16)
-  const int a_row = w * C::MW * 16 + (mi & 1) * 8 + r8, a_kc = mi >> 1;   // scores A: rows = tokens
-  const int v_tok = w * C::MW * 16 + (mi >> 1) * 8 + r8, v_dc = mi & 1;   // P.V A (trans)
+  const int a_row = (mi & 1) * 8 + r8, a_kc = mi >> 1;   // scores A: rows = tokens
+  const int v_tok = (mi >> 1) * 8 + r8, v_dc = mi & 1;   // P.V A (trans): rows = tokens
   const int H = a.H;
   const int dq = C::D_H + a.d_r;
   // columns owned after the hi/lo merge: heads hcol, hcol+1 of this group
@@ -256,15 +310,23 @@ __global__ void __launch_bounds__(C::THREADS, 2)
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
     for (int t0 = j0; t0 < j1; t0 += C::TT, ++k) {
+      if (k % C::W != w) continue;                 // another warp of the group takes it
       const int s = k % C::STAGES;
+#ifdef GVA_TRACE
+      const long long tw0 = clock64();
+#endif
       if (ok) ok = mbar_wait(smem_u32(full + s), (k / C::STAGES) & 1, a.status);
       if (!ok) continue;
+#ifdef GVA_TRACE
+      const long long tw1 = clock64();
+      if (warp == 0 && lane == 0 && a.trace) a.trace[blockIdx.x * 8 + 6] += (unsigned long long)(tw1 - tw0);
+#endif
       if (warp == 0 && lane == 0 && k == 0) trace_mark(a, 3);
       const int nvalid = min(C::TT, j1 - t0);
       uint8_t* st = pipe + s * C::STAGE;
       uint8_t* xg = st + g * C::CB * C::BOX;
       uint8_t* vg = C::GQA ? st + C::XB + g * C::CB * C::BOX : xg;
-      const int r_lo = w * C::MW * 16, r_hi = r_lo + C::MW * 16;   // this warp's rows
+      const int r_lo = 0, r_hi = C::TT;   // this warp's rows: the whole tile
       const bool ragged = nvalid < r_hi;
       if (ragged) {
         // rows past the sequence may hold anything (even NaN): zero this warp's
@@ -320,6 +382,17 @@ __global__ void __launch_bounds__(C::THREADS, 2)
         }
       }
 
+      // ---- V^T fragments for the second product, requested before the softmax so
+      // their shared-memory latency overlaps it
+      uint32_t vf[C::MW][C::KS][4];
+#pragma unroll
+      for (int mm = 0; mm < C::MW; ++mm)
+#pragma unroll
+        for (int md = 0; md < C::KS; ++md)
+          ldsm_x4_t(vg_u + (md >> 2) * C::BOX + (v_tok + mm * 16) * 128 +
+                        ((((md & 3) * 2 + v_dc) ^ r8) << 4),
+                    vf[mm][md][0], vf[mm][md][1], vf[mm][md][2], vf[mm][md][3]);
+
       // ---- online softmax (fp32, base 2); this thread owns heads hcol, hcol+1
       float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
@@ -370,23 +443,22 @@ __global__ void __launch_bounds__(C::THREADS, 2)
           o[nt][md][3] *= al1;
         }
 
-      // ---- O^T += V^T P over this warp's tokens
+      // ---- O^T += V^T P over this warp's tokens (V^T fragments loaded above)
 #pragma unroll
-      for (int mm = 0; mm < C::MW; ++mm) {
-        const int vt = v_tok + mm * 16;
+      for (int mm = 0; mm < C::MW; ++mm)
 #pragma unroll
-        for (int md = 0; md < C::KS; ++md) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(vg_u + (md >> 2) * C::BOX + vt * 128 + ((((md & 3) * 2 + v_dc) ^ r8) << 4), a0,
-                    a1, a2, a3);
+        for (int md = 0; md < C::KS; ++md)
 #pragma unroll
           for (int nt = 0; nt < C::NT; ++nt)
-            mma_bf16(o[nt][md], a0, a1, a2, a3, bp[mm][nt][0], bp[mm][nt][1]);
-        }
-      }
+            mma_bf16(o[nt][md], vf[mm][md][0], vf[mm][md][1], vf[mm][md][2], vf[mm][md][3],
+                     bp[mm][nt][0], bp[mm][nt][1]);
       if (ragged) fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(empty + s));
+#ifdef GVA_TRACE
+      if (warp == 0 && lane == 0 && a.trace)
+        a.trace[blockIdx.x * 8 + 7] += (unsigned long long)(clock64() - tw1);
+#endif
     }
 
     // ---- piece epilogue

@@ -34,13 +34,15 @@ cudaError_t launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, 
   return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
 }
 
+// early_trigger: let the next kernel launch at once (fused step only, see api.cu).
 cudaError_t launch_absorb(const gva_shape_t& sh, const void* q, const void* M, const int* q_pos,
-                          float* q_abs, float c, cudaStream_t st);
+                          float* q_abs, float c, cudaStream_t st, bool early_trigger = false);
 size_t absorb_smem_bytes(const gva_shape_t& sh);
 
 cudaError_t launch_append(const gva_shape_t& sh, int N, const void* v_new, const void* kpe_new,
                           const int* slot, const int* pos, long long num_slots, void* V_cache,
-                          void* kr_cache, int* err_flag, cudaStream_t st);
+                          void* kr_cache, int* err_flag, cudaStream_t st,
+                          bool early_trigger = false);
 
 // CUDA-core split kernel (any dtype / shape within limits).  Returns
 // cudaErrorNotSupported for shapes it is not built for.

@@ -77,8 +77,12 @@ template <typename TQ>
 __global__ void __launch_bounds__(2 * kAbsorbQueries * 32)
     absorb_query_kernel(int B, int H, int d_h, int d_n, int d_r, float c, const TQ* __restrict__ q,
                         const TQ* __restrict__ M, const int* __restrict__ q_pos,
-                        float* __restrict__ q_abs, const RopeTable rt) {
+                        float* __restrict__ q_abs, const RopeTable rt, int early_trigger) {
   extern __shared__ float sm[];
+  // In the fused step the successor (the split kernel) may launch right away: it
+  // waits on this kernel before it reads q_abs, and this kernel waits on the
+  // append before it finishes.
+  if (early_trigger) pdl_trigger();
   const int dq = d_n + d_r, dout = d_h + d_r;
   const int h = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qi = warp % kAbsorbQueries;
@@ -119,7 +123,7 @@ __global__ void __launch_bounds__(2 * kAbsorbQueries * 32)
       for (int k = 0; k < d_n; ++k) acc0 = fmaf(qv[k], to_f32(row[k]), acc0);
     }
     pdl_wait();
-    pdl_trigger();
+    if (!early_trigger) pdl_trigger();
     if (row_ok) o[i] = (acc0 + acc1) * c;
   } else {
     const int half = d_r / 2;
@@ -134,7 +138,7 @@ __global__ void __launch_bounds__(2 * kAbsorbQueries * 32)
                   y2[u]);
     }
     pdl_wait();
-    pdl_trigger();
+    if (!early_trigger) pdl_trigger();
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int p = lane + 32 * u;
@@ -154,8 +158,12 @@ __global__ void append_cache_kernel(int N, int row_elems, int d_r, const T* __re
                                     const T* __restrict__ kpe_new, const int* __restrict__ slot,
                                     const int* __restrict__ pos, long long num_slots,
                                     T* __restrict__ V_cache, T* __restrict__ kr_cache,
-                                    int* __restrict__ err_flag, const RopeTable rt) {
+                                    int* __restrict__ err_flag, const RopeTable rt,
+                                    int early_trigger) {
   constexpr int kVecPerLane = 4;   // rows up to 32*4*16 bytes = 2 KB in registers
+  // In the fused step the absorb kernel may launch right away: it writes nothing
+  // this kernel reads, and it waits on this kernel before it finishes.
+  if (early_trigger) pdl_trigger();
   const int warps = blockDim.x >> 5;
   const int lane = threadIdx.x & 31;
   const long long i = (long long)blockIdx.x * warps + (threadIdx.x >> 5);
@@ -179,7 +187,7 @@ __global__ void append_cache_kernel(int N, int row_elems, int d_r, const T* __re
                 (double)pos[i], rt.inv_freq[p], y1[u], y2[u]);
   }
   pdl_wait();
-  pdl_trigger();
+  if (!early_trigger) pdl_trigger();
   if (active && !ok) {
     if (lane == 0 && err_flag) atomicExch(err_flag, 1);
     return;
@@ -212,7 +220,7 @@ size_t absorb_smem_bytes(const gva_shape_t& sh) {
 }
 
 cudaError_t launch_absorb(const gva_shape_t& sh, const void* q, const void* M, const int* q_pos,
-                          float* q_abs, float c, cudaStream_t st) {
+                          float* q_abs, float c, cudaStream_t st, bool early_trigger) {
   const size_t smem = absorb_smem_bytes(sh);
   const dim3 grid(sh.H, (sh.B + kAbsorbQueries - 1) / kAbsorbQueries, (sh.d_h + 31) / 32);
   const dim3 block(2 * kAbsorbQueries * 32);
@@ -221,17 +229,18 @@ cudaError_t launch_absorb(const gva_shape_t& sh, const void* q, const void* M, c
     auto k = absorb_query_kernel<__nv_bfloat16>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     return launch_pdl(k, grid, block, smem, st, sh.B, sh.H, sh.d_h, sh.d_n, sh.d_r, c,
-                      (const __nv_bfloat16*)q, (const __nv_bfloat16*)M, q_pos, q_abs, rt);
+                      (const __nv_bfloat16*)q, (const __nv_bfloat16*)M, q_pos, q_abs, rt,
+                      early_trigger ? 1 : 0);
   }
   auto k = absorb_query_kernel<float>;
   if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   return launch_pdl(k, grid, block, smem, st, sh.B, sh.H, sh.d_h, sh.d_n, sh.d_r, c, (const float*)q,
-                    (const float*)M, q_pos, q_abs, rt);
+                    (const float*)M, q_pos, q_abs, rt, early_trigger ? 1 : 0);
 }
 
 cudaError_t launch_append(const gva_shape_t& sh, int N, const void* v_new, const void* kpe_new,
                           const int* slot, const int* pos, long long num_slots, void* V_cache,
-                          void* kr_cache, int* err_flag, cudaStream_t st) {
+                          void* kr_cache, int* err_flag, cudaStream_t st, bool early_trigger) {
   const int threads = 256, warps = threads / 32;
   const int grid = (int)(((long long)N + warps - 1) / warps);   // N < 2^31: fits the x grid
   const int row = sh.G * sh.d_h;
@@ -239,10 +248,11 @@ cudaError_t launch_append(const gva_shape_t& sh, int N, const void* v_new, const
   if (sh.cache_dtype == GVA_BF16)
     return launch_pdl(append_cache_kernel<__nv_bfloat16>, dim3(grid), dim3(threads), 0, st, N, row,
                       sh.d_r, (const __nv_bfloat16*)v_new, (const __nv_bfloat16*)kpe_new, slot, pos,
-                      num_slots, (__nv_bfloat16*)V_cache, (__nv_bfloat16*)kr_cache, err_flag, rt);
+                      num_slots, (__nv_bfloat16*)V_cache, (__nv_bfloat16*)kr_cache, err_flag, rt,
+                      early_trigger ? 1 : 0);
   return launch_pdl(append_cache_kernel<float>, dim3(grid), dim3(threads), 0, st, N, row, sh.d_r,
                     (const float*)v_new, (const float*)kpe_new, slot, pos, num_slots,
-                    (float*)V_cache, (float*)kr_cache, err_flag, rt);
+                    (float*)V_cache, (float*)kr_cache, err_flag, rt, early_trigger ? 1 : 0);
 }
 
 }  // namespace gva

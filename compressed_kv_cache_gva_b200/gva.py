@@ -84,6 +84,9 @@ def lib() -> ctypes.CDLL:
         L.gva_decode_attention.argtypes = [SP, P, P, P, P, P, I64, I64, P, P, P, SZ, P]
         L.gqa_decode_attention.restype = ctypes.c_int
         L.gqa_decode_attention.argtypes = [SP, P, P, P, P, P, I64, I64, P, P, P, SZ, P]
+        L.gva_decode_step.restype = ctypes.c_int
+        L.gva_decode_step.argtypes = [SP, P, P, P, I32, P, P, P, P, P, P, I64, P, P, I64, P, P, P, P,
+                                      P, SZ, P]
         L.gva_decode_attention_noalloc.restype = ctypes.c_int
         L.gva_decode_attention_noalloc.argtypes = [SP, P, P, P, P, P, I64, I64, P, P, P]
         _lib = L
@@ -157,6 +160,18 @@ def gqa_decode_attention(shape: Shape, q, K_cache, V_cache, seq_offset, seq_len,
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def decode_step(shape: Shape, q, M, q_pos, v_new, kpe_new, slot, pos, V_cache, kr_cache,
+                seq_offset, seq_len, max_total_tokens: int, q_abs, out, lse=None, err_flag=None,
+                workspace=None, stream=None):
+    """gva_decode_step: append the new tokens, absorb the queries, decode."""
+    _check(lib().gva_decode_step(
+        ctypes.byref(shape), _ptr(q), _ptr(M), _ptr(q_pos), slot.numel(), _ptr(v_new),
+        _ptr(kpe_new), _ptr(slot), _ptr(pos), _ptr(V_cache), _ptr(kr_cache), V_cache.shape[0],
+        _ptr(seq_offset), _ptr(seq_len), int(max_total_tokens), _ptr(q_abs), _ptr(out), _ptr(lse),
+        _ptr(err_flag), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+
+
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -172,4 +187,4 @@ def decode_attention_noalloc(shape: Shape, q_abs, V_cache, kr_cache, seq_offset,
 
 EXPORTS = ["gva_status_string", "gva_last_error", "gva_absorb_query", "gva_append_cache",
            "gva_decode_workspace_size", "gva_decode_attention", "gqa_decode_attention",
-           "gva_decode_attention_noalloc"]
+           "gva_decode_step", "gva_decode_attention_noalloc"]

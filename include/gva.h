@@ -177,6 +177,27 @@ gva_status_t gqa_decode_attention(const gva_shape_t* shape, const void* q, const
                                   size_t ws_bytes, void* stream);
 
 /*
+ * gva_decode_step — one full GVA decode step: gva_append_cache of the n_new new
+ * tokens, gva_absorb_query, then gva_decode_attention, enqueued on `stream` in
+ * that order (onedev.kr review, "How it works" and "What differs": the new
+ * token's value and rotated positional key are cached, the query is absorbed,
+ * content attention reads only the value cache).  Arguments are those of the
+ * three calls; seq_len must already count the new tokens, q_abs is the caller's
+ * [B, H, d_h + d_r] float32 buffer for the absorbed queries, err_flag may be NULL.
+ * Because the append finishes before the decode is launched, the decode starts
+ * streaming the cache while the absorb kernel still runs.  Validation of all three
+ * parts happens before the first launch, except for errors only the append or
+ * absorb checks catch, in which case the earlier parts may have been enqueued.
+ */
+gva_status_t gva_decode_step(const gva_shape_t* shape, const void* q, const void* M,
+                             const int32_t* q_pos, int32_t n_new, const void* v_new,
+                             const void* kpe_new, const int32_t* slot, const int32_t* pos,
+                             void* V_cache, void* kr_cache, int64_t num_slots,
+                             const int32_t* seq_offset, const int32_t* seq_len,
+                             int64_t max_total_tokens, float* q_abs, void* out, float* lse,
+                             int32_t* err_flag, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * gva_decode_attention_noalloc — gva_decode_attention for callers that cannot
  * allocate device memory.  The paper has no counterpart: this is an interface
  * convenience of this library.

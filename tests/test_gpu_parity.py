@@ -235,3 +235,49 @@ def test_shared_kv_gva_equals_gqa():
     out_gqa, lse_gqa, _ = run_gqa(gi, 16, 4, 64, torch.bfloat16)
     assert_close(out_gqa, ref, "bf16", "gqa K=V")
     assert np.max(np.abs(out_gqa - out_gva)) < 1e-3
+
+
+# ------------------------------------------------------------------ fused decode step
+
+@pytest.mark.parametrize("name", ["350m_b8_t4096", "d128_b1_t131072", "tiny_fp32_t64"])
+def test_decode_step_matches_oracle_and_separate_calls(name):
+    """gva_decode_step (append, absorb, decode in one call, decode streaming the
+    cache before absorb finishes) against the oracle's append + decode, and
+    bit-identical to the three separate calls."""
+    wl = WORKLOADS[name]
+    lengths = np.array([300, 65, 1, 1031][:max(1, min(4, wl.B + 3))])
+    di = make_decode_inputs(wl, extra_slots=1, lengths=lengths)
+    V0, K0 = as_f64(di.V), as_f64(di.k_rope)
+    offs = di.seq_offset.numpy()
+    slots = (offs + lengths).astype(np.int32)
+    ap = make_append_inputs(wl, slots, lengths.astype(np.int32))
+    seq_len = torch.from_numpy((lengths + 1).astype(np.int32))
+    q_pos = torch.from_numpy(lengths.astype(np.int32))
+    B = len(lengths)
+    sh = shape_of(di)
+    total = int(seq_len.sum())
+    outs = []
+    for fused in (True, False):
+        V, KR = dev(di.V), dev(di.k_rope)
+        q_abs = torch.empty(B, wl.H, wl.d_h + wl.d_r, dtype=torch.float32, device="cuda")
+        out = torch.empty(B, wl.H, wl.d_h, dtype=torch.float32, device="cuda")
+        lse = torch.empty(B, wl.H, dtype=torch.float32, device="cuda")
+        ws = gva.new_workspace(sh, total)
+        if fused:
+            gva.decode_step(sh, dev(di.q), dev(di.M), dev(q_pos), dev(ap.v_new), dev(ap.kpe_new),
+                            dev(ap.slot), dev(ap.pos), V, KR, dev(di.seq_offset), dev(seq_len), total,
+                            q_abs, out, lse, None, ws)
+        else:
+            gva.append_cache(sh, dev(ap.v_new), dev(ap.kpe_new), dev(ap.slot), dev(ap.pos), V, KR)
+            gva.absorb_query(sh, dev(di.q), dev(di.M), dev(q_pos), q_abs)
+            gva.decode_attention(sh, q_abs, V, KR, dev(di.seq_offset), dev(seq_len), total, out, lse, ws)
+        torch.cuda.synchronize()
+        assert gva.workspace_status(ws) == 0
+        outs.append((out.cpu().numpy(), lse.cpu().numpy()))
+    V_ref, K_ref, _ = oracle.append_cache(V0, K0, as_f64(ap.v_new), as_f64(ap.kpe_new), slots, lengths,
+                                          wl.rope_base, wl.dtype)
+    ref, ref_lse = oracle.gva_decode(as_f64(di.q), as_f64(di.M), q_pos.numpy(), V_ref, K_ref, offs,
+                                     seq_len.numpy(), wl.d_n, wl.d_r, wl.rope_base)
+    assert_close(outs[0][0], ref, wl.dtype, "decode_step")
+    lse_close(outs[0][1], ref_lse)
+    assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
