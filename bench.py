@@ -52,6 +52,10 @@ def parse():
     p.add_argument("--ctas-per-sm", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--split", default="batch", choices=["batch", "sequence"],
+                   help="batch: one independent batch per GPU (weak scaling, default); "
+                        "sequence: one batch, every sequence's cache split across the GPUs "
+                        "(strong scaling, NCCL all-gather + merge)")
     return p.parse_args()
 
 
@@ -189,45 +193,76 @@ def ncu_traffic(kernel_key, workload):
 def run_ours(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    wl = rank_workload(args.workload, rank)
+    split_seq = args.split == "sequence"
+    # sequence split: every rank holds a part of the same batch
+    wl = WORKLOADS[args.workload] if split_seq else rank_workload(args.workload, rank)
     di = make_decode_inputs(wl, extra_slots=1)
     B, H, G, d_h, d_r = len(di.seq_len), wl.H, wl.G, wl.d_h, wl.d_r
     L = di.seq_len.numpy().astype(np.int64)
     row_bytes = cache_row_bytes(wl)
     step_tokens = int((L + 1).sum())                       # history + the appended token
-    step_cache_bytes = step_tokens * row_bytes
-    cache_bytes = di.num_slots * row_bytes
+    step_cache_bytes = step_tokens * row_bytes             # this rank's batch (or whole batch)
+    slots_np = (di.seq_offset.numpy() + L).astype(np.int32)
+    ap = make_append_inputs(wl, slots_np, L.astype(np.int32), seed=7 + (0 if split_seq else rank))
+    app_host = [ap.v_new, ap.kpe_new, ap.slot, ap.pos]
+    V_src, K_src, soff_src = di.V, di.k_rope, di.seq_offset
+    slen_src = torch.from_numpy((L + 1).astype(np.int32))
+    if split_seq:
+        from compressed_kv_cache_gva_b200 import seqsplit
+        V_src, K_src, soff_src, slen_src, start = seqsplit.shard_cache(
+            di.V, di.k_rope, di.seq_offset, slen_src, world, rank)
+        cnt = slen_src.numpy().astype(np.int64)
+        own = (L >= start) & (L < start + cnt)            # new token of sequence b lands here
+        sl = (soff_src.numpy().astype(np.int64) + L - start)[own].astype(np.int32)
+        app_host = [ap.v_new[torch.from_numpy(own)].contiguous(),
+                    ap.kpe_new[torch.from_numpy(own)].contiguous(),
+                    torch.from_numpy(sl), ap.pos[torch.from_numpy(own)].contiguous()]
+    part_tokens = int(slen_src.to(torch.int64).sum())
+    cache_bytes = max(1, V_src.shape[0]) * row_bytes
     R = max(2, math.ceil(3 * L2_BYTES / cache_bytes))
     flags = gva.FLAG_FMA_PATH if args.fma else 0
     sh = gva.make_shape(B, H, G, d_h, wl.d_n, d_r, cache_dtype=wl.torch_dtype, rope_base=wl.rope_base,
                         flags=flags, ctas_per_sm=args.ctas_per_sm)
 
     d = lambda t: t.to(dev).contiguous()
-    Vs = [d(di.V) for _ in range(R)]
-    KRs = [d(di.k_rope) for _ in range(R)]
+    Vs = [d(V_src) for _ in range(R)]
+    KRs = [d(K_src) for _ in range(R)]
     q, M = d(di.q), d(di.M)
-    soff = d(di.seq_offset)
-    slen_step = d(torch.from_numpy((L + 1).astype(np.int32)))
+    soff = d(soff_src)
+    slen_step = d(slen_src)
     qpos = d(di.seq_len)                                    # new token at position L_b
-    slots_np = (di.seq_offset.numpy() + L).astype(np.int32)
-    ap = make_append_inputs(wl, slots_np, L.astype(np.int32), seed=7 + rank)
-    v_new, kpe_new, slot, pos = d(ap.v_new), d(ap.kpe_new), d(ap.slot), d(ap.pos)
+    v_new, kpe_new, slot, pos = (d(t) for t in app_host)
     q_abs = torch.empty(B, H, d_h + d_r, dtype=torch.float32, device=dev)
     out = torch.empty(B, H, d_h, dtype=torch.float32, device=dev)
-    max_total = step_tokens
+    max_total = max(part_tokens, 1)
     ws = gva.new_workspace(sh, max_total, device=dev)
+    merger = None
+    if split_seq:
+        merger = seqsplit.SequenceSplitMerge(sh, world, dev)
+    dec_out = merger.out_part if split_seq else out
+    dec_lse = merger.lse_part if split_seq else None
 
-    def step(c):
-        gva.decode_step(sh, q, M, qpos, v_new, kpe_new, slot, pos, Vs[c], KRs[c], soff, slen_step,
-                        max_total, q_abs, out, None, None, ws)
+    def finish():
+        if split_seq:
+            merger.merge(out)
+
+    def step(c, qq=None, app=None):
+        vv, kk, ss, pp = app if app is not None else (v_new, kpe_new, slot, pos)
+        gva.decode_step(sh, q if qq is None else qq, M, qpos, vv, kk, ss, pp, Vs[c], KRs[c], soff,
+                        slen_step, max_total, q_abs, dec_out, dec_lse, None, ws)
+        finish()
 
     def step_separate(c):
         gva.append_cache(sh, v_new, kpe_new, slot, pos, Vs[c], KRs[c])
         gva.absorb_query(sh, q, M, qpos, q_abs)
-        gva.decode_attention(sh, q_abs, Vs[c], KRs[c], soff, slen_step, max_total, out, None, ws)
+        gva.decode_attention(sh, q_abs, Vs[c], KRs[c], soff, slen_step, max_total, dec_out, dec_lse,
+                             ws)
+        finish()
 
     def decode_only(c):
-        gva.decode_attention(sh, q_abs, Vs[c], KRs[c], soff, slen_step, max_total, out, None, ws)
+        gva.decode_attention(sh, q_abs, Vs[c], KRs[c], soff, slen_step, max_total, dec_out, dec_lse,
+                             ws)
+        finish()
 
     # eager warm-up (initialises the library and the launch attributes)
     for c in range(R):
@@ -311,34 +346,16 @@ def run_ours(args, rank, world, local):
     g_dec = graphs_for(decode_only, K)
     replay(g_dec)
     ms_dec, _, _ = timed(g_dec, K)
-    gi = make_gqa_inputs(wl, extra_slots=1)
-    Kq = [d(gi.K) for _ in range(R)]
-    Vq = [d(gi.V) for _ in range(R)]
-    sh_q = gva.make_shape(B, H, G, d_h, d_h, 0, cache_dtype=wl.torch_dtype, flags=flags,
-                          ctas_per_sm=args.ctas_per_sm)
-    qg = d(gi.q)
-    slen_q = d(torch.from_numpy((gi.seq_len.numpy() + 1).astype(np.int32)))
-    soff_q = d(gi.seq_offset)
-    tot_q = int(gi.seq_len.numpy().astype(np.int64).sum()) + B
-    ws_q = gva.new_workspace(sh_q, tot_q, device=dev)
-    out_q = torch.empty(B, H, d_h, dtype=torch.float32, device=dev)
-
-    def gqa_decode(c):
-        gva.gqa_decode_attention(sh_q, qg, Kq[c], Vq[c], soff_q, slen_q, tot_q, out_q, None, ws_q)
-
-    for c in range(R):
-        gqa_decode(c)
-    g_gqa = graphs_for(gqa_decode, K)
-    replay(g_gqa)
-    ms_gqa, _, _ = timed(g_gqa, K)
-    gqa_bytes = tot_q * 2 * G * d_h * wl.elem_bytes
-    del Kq, Vq
+    ms_gqa = None
+    if not split_seq:
+        ms_gqa, gqa_bytes = run_gqa_comparison(args, wl, B, H, G, d_h, R, flags, d, graphs_for,
+                                               replay, timed, dev)
 
     # end to end through the public API with host buffers: every step copies its
     # inputs (q, new value, new positional key, slot, position) from one pinned
     # host buffer into one device staging buffer, runs the step on views of it,
     # and reads the output back into pinned host memory
-    parts = [di.q, ap.v_new, ap.kpe_new, ap.slot, ap.pos]
+    parts = [di.q] + app_host
     offs_b, nb = [], 0
     for t in parts:
         offs_b.append(nb)
@@ -360,8 +377,7 @@ def run_ours(args, rank, world, local):
 
     def e2e_step(c):
         d_stage.copy_(h_stage, non_blocking=True)
-        gva.decode_step(sh, eq, M, qpos, ev, ek, es, ep, Vs[c], KRs[c], soff, slen_step, max_total,
-                        q_abs, out, None, None, ws)
+        step(c, qq=eq, app=(ev, ek, es, ep))
         h_out.copy_(out, non_blocking=True)
 
     g_e2e = graphs_for(e2e_step, K)
@@ -370,21 +386,25 @@ def run_ours(args, rank, world, local):
 
     hbm_peak, peak_kind = load_peaks()
     ms_step = ms / K
-    value = job_value(step_cache_bytes, K, world, ms)
+    job_ranks = 1 if split_seq else world      # sequence split: one batch for all ranks
+    value = job_value(step_cache_bytes, K, job_ranks, ms)
     dec_s = ms_dec / K * 1e-3
-    alg_dec_bytes = step_cache_bytes + B * H * (d_h + d_r) * 4 + B * H * d_h * 4
+    alg_dec_bytes = part_tokens * row_bytes + B * H * (d_h + d_r) * 4 + B * H * d_h * 4
     achieved = alg_dec_bytes / dec_s / 1e9
     kernel_key = "gva_decode_attention" + ("_fma" if args.fma else "")
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
-        "warmup": W, "ms_per_step": round(ms_step, 6), "higher_is_better": True, "scaling": "weak",
+        "warmup": W, "ms_per_step": round(ms_step, 6), "higher_is_better": True,
+        "scaling": "strong" if split_seq else "weak",
         "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": wl.name, "B": B, "H": H, "G": G, "d_h": d_h, "d_n": wl.d_n, "d_r": d_r,
                    "T": wl.T, "ragged": wl.ragged, "rope_base": wl.rope_base,
                    "tokens_per_step": step_tokens, "cache_bytes_per_step": step_cache_bytes,
                    "l2": f"inputs larger than L2: {R} rotating cache copies, "
                          f"{R * cache_bytes / 2**20:.0f} MiB",
-                   "parallelism": f"weak: {world} independent batch(es), one per GPU",
+                   "parallelism": (f"sequence split: each sequence's cache over {world} GPU(s), "
+                                   "NCCL all-gather of (out, lse) + merge") if split_seq else
+                                  f"weak: {world} independent batch(es), one per GPU",
                    "step": "gva_decode_step: append + absorb + decode (split + combine)",
                    "graphs": "CUDA graphs",
                    "decode_path": "fma" if args.fma else "tensor"},
@@ -392,7 +412,7 @@ def run_ours(args, rank, world, local):
         "ms_per_step_separate_calls": round(ms_sep / K, 6),
         "pct_hbm_peak": {"of_measured": round(value / world / hbm_peak, 4),
                          "of_nominal_8TBs": round(value / world / NOMINAL_HBM_GBS, 4)},
-        "gqa_comparison": {
+        "gqa_comparison": None if ms_gqa is None else {
             "gva_decode_steps_per_s": round(K / (ms_dec * 1e-3), 1),
             "gqa_decode_steps_per_s": round(K / (ms_gqa * 1e-3), 1),
             "decode_speedup_vs_gqa": round(ms_gqa / ms_dec, 4),
@@ -406,13 +426,38 @@ def run_ours(args, rank, world, local):
                      "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                      "alg_bytes_per_launch": alg_dec_bytes, "us_per_launch": round(dec_s * 1e6, 3),
                      "traffic": ncu_traffic(kernel_key, wl.name)},
-        "e2e": {"value": round(job_value(step_cache_bytes, K, world, ms_e2e), 2), "unit": "GB/s",
+        "e2e": {"value": round(job_value(step_cache_bytes, K, job_ranks, ms_e2e), 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(ms_e2e / K, 6)},
-        "gpu_launches": 4 * K,
+        "gpu_launches": (5 if split_seq else 4) * K,
         "clocks": clocks,
     }
     return res, di
+
+
+def run_gqa_comparison(args, wl, B, H, G, d_h, R, flags, d, graphs_for, replay, timed, dev):
+    """Same-shape GQA decode (K and V cache) timed like the GVA decode."""
+    gi = make_gqa_inputs(wl, extra_slots=1)
+    Kq = [d(gi.K) for _ in range(R)]
+    Vq = [d(gi.V) for _ in range(R)]
+    sh_q = gva.make_shape(B, H, G, d_h, d_h, 0, cache_dtype=wl.torch_dtype, flags=flags,
+                          ctas_per_sm=args.ctas_per_sm)
+    qg = d(gi.q)
+    slen_q = d(torch.from_numpy((gi.seq_len.numpy() + 1).astype(np.int32)))
+    soff_q = d(gi.seq_offset)
+    tot_q = int(gi.seq_len.numpy().astype(np.int64).sum()) + B
+    ws_q = gva.new_workspace(sh_q, tot_q, device=dev)
+    out_q = torch.empty(B, H, d_h, dtype=torch.float32, device=dev)
+
+    def gqa_decode(c):
+        gva.gqa_decode_attention(sh_q, qg, Kq[c], Vq[c], soff_q, slen_q, tot_q, out_q, None, ws_q)
+
+    for c in range(R):
+        gqa_decode(c)
+    g_gqa = graphs_for(gqa_decode, args.steps)
+    replay(g_gqa)
+    ms_gqa, _, _ = timed(g_gqa, args.steps)
+    return ms_gqa, tot_q * 2 * G * d_h * wl.elem_bytes
 
 
 # ----------------------------------------------------------------------------- oracle arm

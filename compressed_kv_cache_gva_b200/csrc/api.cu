@@ -357,6 +357,20 @@ gva_status_t gva_decode_step(const gva_shape_t* shape, const void* q, const void
                        /*prefetch=*/true, slot, n_new);
 }
 
+gva_status_t gva_merge_states(const gva_shape_t* shape, int32_t R, const float* outs,
+                              const float* lses, void* out, float* lse, void* stream) {
+  gva_status_t s = check_shape(shape, true);
+  if (s != GVA_OK) return s;
+  if (R < 1 || R > 1024) return fail(GVA_ERR_INVALID_ARG, "R=%d outside [1,1024]", R);
+  if (shape->B == 0) return GVA_OK;
+  if (!outs || !lses || !out) return fail(GVA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned16(outs) || !aligned16(lses) || !aligned16(out) || (lse && !aligned16(lse)))
+    return fail(GVA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  cudaError_t e = gva::launch_merge_states(*shape, R, outs, lses, out, lse,
+                                           static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GVA_OK : cuda_fail(e, "merge launch");
+}
+
 gva_status_t gqa_decode_attention(const gva_shape_t* shape, const void* q, const void* K_cache,
                                   const void* V_cache, const int32_t* seq_offset,
                                   const int32_t* seq_len, int64_t max_total_tokens, int64_t num_slots,

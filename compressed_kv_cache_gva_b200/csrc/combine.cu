@@ -150,4 +150,47 @@ cudaError_t launch_combine(const gva_shape_t& sh, const DecodeArgs& a, void* out
   return launch_pdl(combine_kernel<float>, grid, dim3(32 * npg), 0, st, a, (float*)out, lse);
 }
 
+// Merge of R normalised attention states of the same queries over disjoint parts
+// of each sequence's cache (one part per GPU when a sequence is split across
+// GPUs): lse = log sum_r exp(lse_r), out = sum_r exp(lse_r - lse) out_r.
+// One CTA per (sequence, head); threads over d_h.
+template <typename TO>
+__global__ void __launch_bounds__(128)
+    merge_states_kernel(int R, int BH, int d_h, const float* __restrict__ outs,
+                        const float* __restrict__ lses, TO* __restrict__ out,
+                        float* __restrict__ lse) {
+  const int bh = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  float mx = -INFINITY;
+  for (int r = 0; r < R; ++r) mx = fmaxf(mx, lses[(size_t)r * BH + bh]);
+  float z = 0.f;
+  if (mx != -INFINITY)
+    for (int r = 0; r < R; ++r) z += ex2((lses[(size_t)r * BH + bh] - mx) * kLog2e);
+  for (int d = threadIdx.x; d < d_h; d += blockDim.x) {
+    float acc = 0.f;
+    if (mx != -INFINITY)
+      for (int r = 0; r < R; ++r) {
+        const float l = lses[(size_t)r * BH + bh];
+        if (l == -INFINITY) continue;              // an empty part contributes nothing
+        acc = fmaf(ex2((l - mx) * kLog2e), outs[((size_t)r * BH + bh) * d_h + d], acc);
+      }
+    const float v = mx != -INFINITY ? acc / z : 0.f;
+    if constexpr (sizeof(TO) == 2) out[(size_t)bh * d_h + d] = __float2bfloat16_rn(v);
+    else out[(size_t)bh * d_h + d] = v;
+  }
+  if (threadIdx.x == 0 && lse) lse[bh] = mx != -INFINITY ? mx + log2f(z) * kLn2 : -INFINITY;
+}
+
+cudaError_t launch_merge_states(const gva_shape_t& sh, int R, const float* outs, const float* lses,
+                                void* out, float* lse, cudaStream_t st) {
+  const int BH = sh.B * sh.H;
+  const int threads = sh.d_h >= 128 ? 128 : ((sh.d_h + 31) / 32) * 32;
+  if (sh.out_dtype == GVA_BF16)
+    return launch_pdl(merge_states_kernel<__nv_bfloat16>, dim3(BH), dim3(threads), 0, st, R, BH,
+                      sh.d_h, outs, lses, (__nv_bfloat16*)out, lse);
+  return launch_pdl(merge_states_kernel<float>, dim3(BH), dim3(threads), 0, st, R, BH, sh.d_h,
+                    outs, lses, (float*)out, lse);
+}
+
 }  // namespace gva

@@ -58,6 +58,10 @@ cudaError_t launch_decode_mma(const gva_shape_t& sh, bool gqa, DecodeArgs& a,
                               const CUtensorMap& tm_x, const CUtensorMap& tm_v,
                               const CUtensorMap& tm_kr, cudaStream_t st);
 
+// Merge of R normalised states (out, lse) of the same queries (sequence split).
+cudaError_t launch_merge_states(const gva_shape_t& sh, int R, const float* outs, const float* lses,
+                                void* out, float* lse, cudaStream_t st);
+
 // Log-sum-exp combine of the partials into the output.
 cudaError_t launch_combine(const gva_shape_t& sh, const DecodeArgs& a, void* out, float* lse,
                            cudaStream_t st);

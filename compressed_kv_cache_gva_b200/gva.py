@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
         L.gva_decode_step.restype = ctypes.c_int
         L.gva_decode_step.argtypes = [SP, P, P, P, I32, P, P, P, P, P, P, I64, P, P, I64, P, P, P, P,
                                       P, SZ, P]
+        L.gva_merge_states.restype = ctypes.c_int
+        L.gva_merge_states.argtypes = [SP, I32, P, P, P, P, P]
         L.gva_decode_attention_noalloc.restype = ctypes.c_int
         L.gva_decode_attention_noalloc.argtypes = [SP, P, P, P, P, P, I64, I64, P, P, P]
         _lib = L
@@ -172,6 +174,12 @@ def decode_step(shape: Shape, q, M, q_pos, v_new, kpe_new, slot, pos, V_cache, k
         _stream(stream)))
 
 
+def merge_states(shape: Shape, outs, lses, out, lse=None, stream=None):
+    """gva_merge_states: outs [R,B,H,d_h] float32, lses [R,B,H] float32."""
+    _check(lib().gva_merge_states(ctypes.byref(shape), outs.shape[0], _ptr(outs), _ptr(lses),
+                                  _ptr(out), _ptr(lse), _stream(stream)))
+
+
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -187,4 +195,4 @@ def decode_attention_noalloc(shape: Shape, q_abs, V_cache, kr_cache, seq_offset,
 
 EXPORTS = ["gva_status_string", "gva_last_error", "gva_absorb_query", "gva_append_cache",
            "gva_decode_workspace_size", "gva_decode_attention", "gqa_decode_attention",
-           "gva_decode_step", "gva_decode_attention_noalloc"]
+           "gva_decode_step", "gva_merge_states", "gva_decode_attention_noalloc"]

@@ -198,6 +198,23 @@ gva_status_t gva_decode_step(const gva_shape_t* shape, const void* q, const void
                              int32_t* err_flag, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * gva_merge_states — merge R attention states of the same queries computed over
+ * disjoint parts of each sequence's cache, e.g. one part per GPU when one long
+ * sequence's cache is split across GPUs.  The pages have no counterpart (they
+ * run no long-context or multi-GPU test: onedev.kr review, "Premises and
+ * limits"); the merge is the exact decomposition of softmax attention:
+ *   lse = log sum_r exp(lse_r),   out = sum_r exp(lse_r - lse) * out_r.
+ *
+ *   outs  device [R, B, H, d_h] float32  normalised outputs of the R parts
+ *   lses  device [R, B, H]      float32  their natural-log lse (-inf: empty part,
+ *                                        whose output is ignored)
+ *   out   device [B, H, d_h] out_dtype; lse device [B, H] float32 or NULL
+ *   Only shape->B, H, d_h and out_dtype are used.  All-empty -> 0 and -inf.
+ */
+gva_status_t gva_merge_states(const gva_shape_t* shape, int32_t R, const float* outs,
+                              const float* lses, void* out, float* lse, void* stream);
+
+/*
  * gva_decode_attention_noalloc — gva_decode_attention for callers that cannot
  * allocate device memory.  The paper has no counterpart: this is an interface
  * convenience of this library.
