@@ -33,7 +33,8 @@ sys.path.insert(0, ROOT)
 
 from compressed_kv_cache_gva_b200 import gva  # noqa: E402
 from compressed_kv_cache_gva_b200.synth import (WORKLOADS, make_append_inputs,  # noqa: E402
-                                                make_decode_inputs, make_gqa_inputs)
+                                                make_decode_inputs, make_gqa_inputs,
+                                                make_multi_queries)
 
 METRIC = "GVA decode cache GB/s & %HBM peak (1xB200); decode steps/s vs same-shape GQA"
 DEFAULT_WORKLOAD = "350m_b8_t4096"
@@ -346,6 +347,10 @@ def run_ours(args, rank, world, local):
     g_dec = graphs_for(decode_only, K)
     replay(g_dec)
     ms_dec, _, _ = timed(g_dec, K)
+    multi = None
+    if not args.fma and not split_seq and (H // G) * 2 in (4, 8):
+        multi = time_multi_token(sh, wl, di, 2, Vs, KRs, soff, slen_step, max_total, M, R, d,
+                                 graphs_for, replay, timed, K, dev, row_bytes, part_tokens, ms_dec)
     ms_gqa = None
     if not split_seq:
         ms_gqa, gqa_bytes = run_gqa_comparison(args, wl, B, H, G, d_h, R, flags, d, graphs_for,
@@ -429,10 +434,43 @@ def run_ours(args, rank, world, local):
         "e2e": {"value": round(job_value(step_cache_bytes, K, job_ranks, ms_e2e), 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(ms_e2e / K, 6)},
+        "multi_token": multi,
         "gpu_launches": (5 if split_seq else 4) * K,
         "clocks": clocks,
     }
     return res, di
+
+
+def time_multi_token(sh, wl, di, Q, Vs, KRs, soff, slen, max_total, M, R, d, graphs_for, replay,
+                     timed, K, dev, row_bytes, part_tokens, ms_dec):
+    """Q new tokens per sequence decoded together (causal among them), as in
+    speculative-decoding verification: one gva_decode_attention_multi call on the
+    same caches, timed like the single-token decode."""
+    B, H, d_h, d_r = len(di.seq_len), wl.H, wl.d_h, wl.d_r
+    q = make_multi_queries(wl, B, Q)
+    L = di.seq_len.numpy().astype(np.int64) + 1
+    qpos = torch.from_numpy(np.stack([L - Q + i for i in range(Q)], 1).astype(np.int32))
+    sh_q = gva.make_shape(B * Q, H, wl.G, d_h, wl.d_n, d_r, cache_dtype=wl.torch_dtype,
+                          rope_base=wl.rope_base)
+    q_abs = torch.empty(B, Q, H, d_h + d_r, dtype=torch.float32, device=dev)
+    gva.absorb_query(sh_q, d(q.reshape(B * Q, H, -1)), M, d(qpos.reshape(-1)), q_abs)
+    ws = torch.zeros(gva.decode_workspace_size_multi(sh, Q, max_total), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty(B, Q, H, d_h, dtype=torch.float32, device=dev)
+
+    def call(c):
+        gva.decode_attention_multi(sh, Q, q_abs, Vs[c], KRs[c], soff, slen, max_total, out, None, ws)
+
+    for c in range(R):
+        call(c)
+    gs = graphs_for(call, K)
+    replay(gs)
+    ms, _, _ = timed(gs, K)
+    assert gva.workspace_status(ws) == 0, "device status word set"
+    s = ms / K * 1e-3
+    alg = part_tokens * row_bytes + B * Q * H * (d_h + d_r) * 4 + B * Q * H * d_h * 4
+    return {"n_query": Q, "call": "gva_decode_attention_multi", "us_per_call": round(s * 1e6, 3),
+            "alg_GBs": round(alg / s / 1e9, 2), "time_vs_single_token_decode": round(ms / ms_dec, 4)}
 
 
 def run_gqa_comparison(args, wl, B, H, G, d_h, R, flags, d, graphs_for, replay, timed, dev):

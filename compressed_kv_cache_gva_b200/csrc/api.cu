@@ -136,10 +136,15 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
                            const int32_t* seq_len, int64_t max_total_tokens, int64_t num_slots,
                            void* out, float* lse, void* workspace, size_t ws_bytes, void* stream,
                            bool prefetch = false, const int32_t* new_slots = nullptr,
-                           int n_new = 0) {
+                           int n_new = 0, int nq = 1) {
   gva_status_t s = check_shape(shp, gqa);
   if (s != GVA_OK) return s;
-  const gva_shape_t& sh = *shp;
+  if (nq < 1 || nq > 64) return fail(GVA_ERR_INVALID_ARG, "n_query=%d outside [1,64]", nq);
+  // nq query tokens per sequence run as nq * H/G columns per value group: the
+  // kernels and the workspace see H * nq heads, the queries see H heads each
+  gva_shape_t shv = *shp;
+  shv.H = shp->H * nq;
+  const gva_shape_t& sh = shv;
   if (sh.B == 0) return GVA_OK;
   if (!q || !X || !Vv || !seq_offset || !seq_len || !out || !workspace)
     return fail(GVA_ERR_INVALID_ARG, "a required pointer is NULL");
@@ -157,12 +162,16 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
                 sh.G * sh.d_h * e, gqa ? 0 : sh.d_r * e);
   Plan p;
   if ((s = plan_decode(sh, gqa, max_total_tokens, &p)) != GVA_OK) return s;
+  if (nq > 1 && !p.mma)
+    return fail(GVA_ERR_UNSUPPORTED, "several query tokens need the tensor-core kernel "
+                "(bf16 cache, (H/G)*n_query in {4, 8}, d_h in {64, 128})");
   if (ws_bytes < p.ws.total)
     return fail(GVA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, p.ws.total);
 
   gva::DecodeArgs a{};
   a.B = sh.B;
-  a.H = sh.H;
+  a.H = shp->H;
+  a.nq = nq;
   a.G = sh.G;
   a.d_h = sh.d_h;
   a.d_r = gqa ? 0 : sh.d_r;
@@ -216,6 +225,7 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
                   sh.d_h, sh.d_r);
   }
   if (err != cudaSuccess) return cuda_fail(err, "decode split kernel launch");
+  a.H = sh.H;   // the combine sees the nq * H heads of the partials
   err = gva::launch_combine(sh, a, out, lse, st);
   if (err != cudaSuccess) return cuda_fail(err, "combine kernel launch");
   return GVA_OK;
@@ -355,6 +365,25 @@ gva_status_t gva_decode_step(const gva_shape_t* shape, const void* q, const void
   return decode_common(shape, false, q_abs, V_cache, V_cache, kr_cache, seq_offset, seq_len,
                        max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream,
                        /*prefetch=*/true, slot, n_new);
+}
+
+size_t gva_decode_workspace_size_multi(const gva_shape_t* shape, int32_t n_query,
+                                       int64_t max_total_tokens) {
+  if (!shape || n_query < 1 || n_query > 64) return 0;
+  gva_shape_t shv = *shape;
+  shv.H = shape->H * n_query;
+  return gva_decode_workspace_size(&shv, max_total_tokens);
+}
+
+gva_status_t gva_decode_attention_multi(const gva_shape_t* shape, int32_t n_query,
+                                        const float* q_abs, const void* V_cache,
+                                        const void* kr_cache, const int32_t* seq_offset,
+                                        const int32_t* seq_len, int64_t max_total_tokens,
+                                        int64_t num_slots, void* out, float* lse,
+                                        void* workspace, size_t ws_bytes, void* stream) {
+  return decode_common(shape, false, q_abs, V_cache, V_cache, kr_cache, seq_offset, seq_len,
+                       max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream, false,
+                       nullptr, 0, n_query);
 }
 
 gva_status_t gva_merge_states(const gva_shape_t* shape, int32_t R, const float* outs,

@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(1024)
 #pragma unroll
     for (int u = 0; u < kCombinePieces; ++u) {
       if (c0 + u * npg >= n) break;
+      if (e[u].x == -INFINITY) continue;          // piece past this query's causal limit
       const float mn = fmaxf(m, e[u].x);
       const float f = ex2(m - mn), w = ex2(e[u].x - mn);
       l = l * f + w * e[u].y;
@@ -121,12 +122,12 @@ __global__ void __launch_bounds__(1024)
     O = fmaf(f, sm_o[u][lane], O);
   }
   if (col) {
-    const float v = n > 0 ? O / L : 0.f;
+    const float v = L > 0.f ? O / L : 0.f;
     if constexpr (sizeof(TO) == 2) out[((size_t)b * H + h) * d_h + d] = __float2bfloat16_rn(v);
     else out[((size_t)b * H + h) * d_h + d] = v;
   }
   if (lane == 0 && blockIdx.z == 0 && lse)
-    lse[(size_t)b * H + h] = n > 0 ? (M + log2f(L)) * kLn2 : -INFINITY;
+    lse[(size_t)b * H + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
 #ifdef GVA_TRACE
   if (a.trace && tid == 0 && cid < 16384) {
     unsigned long long tt;

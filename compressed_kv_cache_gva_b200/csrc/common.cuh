@@ -56,6 +56,7 @@ struct DecodeArgs {
   int2* meta;                // per sequence: (first partial slot, number of pieces)
   float2* part_ml;           // [P][H] (running max, running sum), base-2
   float* part_o;             // [P][H][d_h] un-normalised output
+  int nq;                    // query tokens per sequence (causal among them), >= 1
   int grid;                  // CTAs of the split kernel
   int tile;                  // span granularity in tokens
   int prefetch;              // stream the cache before the PDL wait (fused step only), except

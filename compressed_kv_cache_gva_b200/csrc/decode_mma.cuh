@@ -228,10 +228,16 @@ __global__ void __launch_bounds__(C::THREADS, 2)
   // ldmatrix row/chunk owned by this lane (see the fragment layouts of m16n8k16)
   const int a_row = (mi & 1) * 8 + r8, a_kc = mi >> 1;   // scores A: rows = tokens
   const int v_tok = (mi >> 1) * 8 + r8, v_dc = mi & 1;   // P.V A (trans): rows = tokens
-  const int H = a.H;
+  const int H = a.H;                  // query heads
+  const int hpr = a.H / a.G;          // query heads per group; C::HPG = hpr * nq columns
+  const int Hp = a.H * a.nq;          // heads of the partials and the output: [query][head]
   const int dq = C::D_H + a.d_r;
-  // columns owned after the hi/lo merge: heads hcol, hcol+1 of this group
+  // columns owned after the hi/lo merge: hcol, hcol+1 of this group.  Column c
+  // is query c / hpr of the sequence's nq new tokens and head g*hpr + c % hpr.
   const int hcol = (2 * t) & (C::HPG - 1);
+  const int qi0 = hcol / hpr, qi1 = (hcol + 1) / hpr;   // differ only when H/G is odd
+  const int phead0 = qi0 * H + g * hpr + hcol % hpr;
+  const int phead1 = qi1 * H + g * hpr + (hcol + 1) % hpr;
   const bool lo_half = (C::HPG == 4) && (t >= 2);
   float* mg_ml = merge + g * (C::MERGE_ML + C::MERGE_O);
   float* mg_o = mg_ml + C::MERGE_ML;
@@ -247,13 +253,13 @@ __global__ void __launch_bounds__(C::THREADS, 2)
     uint32_t qr[C::NT][C::RS > 0 ? C::RS : 1][2];
 #pragma unroll
     for (int nt = 0; nt < C::NT; ++nt) {
-      const int hl = C::HPG == 8 ? gq : (gq & 3);
+      const int hl = C::HPG == 8 ? gq : (gq & 3);     // column within the group
       const bool lo = C::HPG == 8 ? (nt == 1) : (gq >= 4);
-      const int head = g * C::HPG + hl;
+      const int vq = hl / hpr, head = g * hpr + hl % hpr;
       float v[C::KS][4];
       float wv[C::RS > 0 ? C::RS : 1][4];
       if constexpr (!C::GQA) {
-        const float* qrow = a.q_abs + ((size_t)b * H + head) * dq;
+        const float* qrow = a.q_abs + (((size_t)b * a.nq + vq) * H + head) * dq;
 #pragma unroll
         for (int ks = 0; ks < C::KS; ++ks) {
           const int k0 = ks * 16 + 2 * t;
@@ -308,6 +314,10 @@ __global__ void __launch_bounds__(C::THREADS, 2)
 #pragma unroll
         for (int e = 0; e < 4; ++e) o[nt][md][e] = 0.f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    // causal limits of this thread's two columns: the nq new tokens sit at
+    // positions L-nq .. L-1 and query i sees the cache up to its own position
+    const int lim0 = (prefix[b + 1] - prefix[b]) - a.nq + qi0;
+    const int lim1 = lim0 + (qi1 - qi0);
 
     for (int t0 = j0; t0 < j1; t0 += C::TT, ++k) {
       if (k % C::W != w) continue;                 // another warp of the group takes it
@@ -378,7 +388,7 @@ __global__ void __launch_bounds__(C::THREADS, 2)
             x += __shfl_xor_sync(0xffffffffu, x, 2);
           }
           const int r = r_lo + mm * 16 + gq + (e >= 2 ? 8 : 0);
-          sc[mm][e] = r < nvalid ? x : -INFINITY;
+          sc[mm][e] = (r < nvalid && t0 + r <= ((e & 1) ? lim1 : lim0)) ? x : -INFINITY;
         }
       }
 
@@ -482,14 +492,17 @@ __global__ void __launch_bounds__(C::THREADS, 2)
         M0 = fmaxf(M0, mg_ml[(u * 4 + t) * 4 + 0]);
         M1 = fmaxf(M1, mg_ml[(u * 4 + t) * 4 + 1]);
       }
+      // a column may have no visible token in this piece (all past its causal
+      // limit): keep it at (-inf, 0) instead of forming -inf - -inf
+      const float Ms0 = M0 == -INFINITY ? 0.f : M0, Ms1 = M1 == -INFINITY ? 0.f : M1;
       float L0 = 0.f, L1 = 0.f;
 #pragma unroll
       for (int u = 0; u < C::W; ++u) {
         const float* e = mg_ml + (u * 4 + t) * 4;
-        L0 += e[2] * ex2(e[0] - M0);
-        L1 += e[3] * ex2(e[1] - M1);
+        L0 += e[2] * ex2(e[0] - Ms0);
+        L1 += e[3] * ex2(e[1] - Ms1);
       }
-      const float f0 = ex2(m0 - M0), f1 = ex2(m1 - M1);
+      const float f0 = ex2(m0 - Ms0), f1 = ex2(m1 - Ms1);
 #pragma unroll
       for (int nt = 0; nt < C::NT; ++nt)
 #pragma unroll
@@ -538,9 +551,8 @@ __global__ void __launch_bounds__(C::THREADS, 2)
       }
     if (ok && (C::HPG == 8 || t < 2)) {
       const size_t slot = (size_t)blockIdx.x + b;
-      const int h0 = g * C::HPG + hcol;
-      float* po0 = a.part_o + (slot * H + h0) * C::D_H;
-      float* po1 = po0 + C::D_H;
+      float* po0 = a.part_o + (slot * Hp + phead0) * C::D_H;
+      float* po1 = a.part_o + (slot * Hp + phead1) * C::D_H;
 #pragma unroll
       for (int md = 0; md < C::KS; ++md) {
         const int d = md * 16 + gq;
@@ -550,8 +562,8 @@ __global__ void __launch_bounds__(C::THREADS, 2)
         po1[d + 8] = o[0][md][3];
       }
       if (gq == 0) {
-        a.part_ml[slot * H + h0] = make_float2(m0, l0);
-        a.part_ml[slot * H + h0 + 1] = make_float2(m1, l1);
+        a.part_ml[slot * Hp + phead0] = make_float2(m0, l0);
+        a.part_ml[slot * Hp + phead1] = make_float2(m1, l1);
       }
     }
     if (warp == 0 && lane == 0) trace_mark(a, 5);

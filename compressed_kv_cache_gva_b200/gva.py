@@ -87,6 +87,10 @@ def lib() -> ctypes.CDLL:
         L.gva_decode_step.restype = ctypes.c_int
         L.gva_decode_step.argtypes = [SP, P, P, P, I32, P, P, P, P, P, P, I64, P, P, I64, P, P, P, P,
                                       P, SZ, P]
+        L.gva_decode_workspace_size_multi.restype = SZ
+        L.gva_decode_workspace_size_multi.argtypes = [SP, I32, I64]
+        L.gva_decode_attention_multi.restype = ctypes.c_int
+        L.gva_decode_attention_multi.argtypes = [SP, I32, P, P, P, P, P, I64, I64, P, P, P, SZ, P]
         L.gva_merge_states.restype = ctypes.c_int
         L.gva_merge_states.argtypes = [SP, I32, P, P, P, P, P]
         L.gva_decode_attention_noalloc.restype = ctypes.c_int
@@ -174,6 +178,22 @@ def decode_step(shape: Shape, q, M, q_pos, v_new, kpe_new, slot, pos, V_cache, k
         _stream(stream)))
 
 
+def decode_workspace_size_multi(shape: Shape, n_query: int, max_total_tokens: int) -> int:
+    return int(lib().gva_decode_workspace_size_multi(ctypes.byref(shape), int(n_query),
+                                                     int(max_total_tokens)))
+
+
+def decode_attention_multi(shape: Shape, n_query: int, q_abs, V_cache, kr_cache, seq_offset,
+                           seq_len, max_total_tokens: int, out, lse=None, workspace=None,
+                           stream=None):
+    """gva_decode_attention_multi: n_query causal query tokens per sequence."""
+    _check(lib().gva_decode_attention_multi(
+        ctypes.byref(shape), int(n_query), _ptr(q_abs), _ptr(V_cache), _ptr(kr_cache),
+        _ptr(seq_offset), _ptr(seq_len), int(max_total_tokens), V_cache.shape[0], _ptr(out),
+        _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+
+
 def merge_states(shape: Shape, outs, lses, out, lse=None, stream=None):
     """gva_merge_states: outs [R,B,H,d_h] float32, lses [R,B,H] float32."""
     _check(lib().gva_merge_states(ctypes.byref(shape), outs.shape[0], _ptr(outs), _ptr(lses),
@@ -195,4 +215,5 @@ def decode_attention_noalloc(shape: Shape, q_abs, V_cache, kr_cache, seq_offset,
 
 EXPORTS = ["gva_status_string", "gva_last_error", "gva_absorb_query", "gva_append_cache",
            "gva_decode_workspace_size", "gva_decode_attention", "gqa_decode_attention",
-           "gva_decode_step", "gva_merge_states", "gva_decode_attention_noalloc"]
+           "gva_decode_step", "gva_merge_states", "gva_decode_workspace_size_multi",
+           "gva_decode_attention_multi", "gva_decode_attention_noalloc"]

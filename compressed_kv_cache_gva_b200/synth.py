@@ -196,3 +196,11 @@ def make_gqa_inputs(wl: Workload, extra_slots: int = 0,
 def as_f64(t: torch.Tensor) -> np.ndarray:
     """Exact widening of a stored tensor to float64 for the oracle."""
     return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+def make_multi_queries(wl: Workload, B: int, n_query: int, seed: int = 2) -> torch.Tensor:
+    """Queries of n_query new tokens per sequence, [B, n_query, H, d_n + d_r],
+    float32 standard normals rounded to the workload's storage type."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, n_query, wl.H, wl.d_n + wl.d_r), dtype=np.float32)
+    return _round(q, wl.dtype)

@@ -198,6 +198,33 @@ gva_status_t gva_decode_step(const gva_shape_t* shape, const void* q, const void
                              int32_t* err_flag, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * gva_decode_attention_multi — decode of n_query new tokens per sequence at once
+ * (e.g. verifying draft tokens in speculative decoding), causal among them: the
+ * new tokens are already appended and occupy positions L-n_query .. L-1 of each
+ * sequence (L = seq_len[b]); query i attends cache positions 0 .. L-n_query+i.
+ * Same absorbed route as gva_decode_attention (onedev.kr review, "How it works"
+ * and "What differs"); each cache tile is read once for all queries and heads of
+ * its group.
+ *
+ *   q_abs  device [B, n_query, H, d_h + d_r] float32: gva_absorb_query run on the
+ *          B*n_query query tokens (shape->B = B*n_query, q_pos = their positions)
+ *   out    device [B, n_query, H, d_h] out_dtype; lse device [B, n_query, H] or NULL
+ *   workspace: gva_decode_workspace_size_multi(shape, n_query, max_total_tokens)
+ *   Other arguments as gva_decode_attention.  Built for bf16 caches with
+ *   (H/G)*n_query in {4, 8} and d_h in {64, 128} (else GVA_ERR_UNSUPPORTED);
+ *   n_query = 1 is gva_decode_attention.
+ */
+size_t gva_decode_workspace_size_multi(const gva_shape_t* shape, int32_t n_query,
+                                       int64_t max_total_tokens);
+
+gva_status_t gva_decode_attention_multi(const gva_shape_t* shape, int32_t n_query,
+                                        const float* q_abs, const void* V_cache,
+                                        const void* kr_cache, const int32_t* seq_offset,
+                                        const int32_t* seq_len, int64_t max_total_tokens,
+                                        int64_t num_slots, void* out, float* lse,
+                                        void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * gva_merge_states — merge R attention states of the same queries computed over
  * disjoint parts of each sequence's cache, e.g. one part per GPU when one long
  * sequence's cache is split across GPUs.  The pages have no counterpart (they

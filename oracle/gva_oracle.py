@@ -248,3 +248,25 @@ def gqa_decode(q: np.ndarray, K: np.ndarray, V: np.ndarray, seq_offset: np.ndarr
         s = (K[o0:o0 + L, g, :] @ q[b, h]) * scale
         out[b, h], lse[b, h] = _softmax_attend(s, V[o0:o0 + L, g, :])
     return out, lse
+
+
+def gva_decode_multi(q: np.ndarray, M: np.ndarray, q_pos: np.ndarray, V: np.ndarray,
+                     k_rope: np.ndarray, seq_offset: np.ndarray, seq_len: np.ndarray, d_n: int,
+                     d_r: int, base: float, scale: Optional[float] = None):
+    """Decode of Q new tokens per sequence at once, causal among them.
+
+    q [B, Q, H, d_n + d_r], q_pos [B, Q].  The Q new tokens are the last Q cache
+    rows of each sequence (positions L-Q .. L-1, L = seq_len[b]); query i attends
+    rows 0 .. L-Q+i, i.e. exactly what a one-token decode at that point of the
+    sequence would see.  Returns (out [B,Q,H,d_h], lse [B,Q,H])."""
+    q = np.asarray(q, dtype=np.float64)
+    B, Q = q.shape[0], q.shape[1]
+    L = np.asarray(seq_len, dtype=np.int64)
+    outs, lses = [], []
+    for i in range(Q):
+        Li = np.maximum(L - Q + i + 1, 0)
+        o, l = gva_decode(q[:, i], M, np.asarray(q_pos)[:, i], V, k_rope, seq_offset, Li, d_n, d_r,
+                          base, scale=scale)
+        outs.append(o)
+        lses.append(l)
+    return np.stack(outs, axis=1), np.stack(lses, axis=1)

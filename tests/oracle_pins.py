@@ -255,6 +255,32 @@ def check_append(orc):
     assert np.max(np.abs(K1[2] - orc.rope(k[0], 5.0, 10000.0))) < 1e-6         # float32 storage
 
 
+def check_multi_query_causal(orc):
+    """Several new tokens decoded together: one query reduces to the one-token
+    decode; the last query sees the whole cache; query i does not see rows after
+    its own position (changing them leaves it unchanged but moves later queries)."""
+    rng = np.random.default_rng(21)
+    c = _rand_case(rng, B=2, H=4, G=2, d_h=8, d_n=6, d_r=4, lens=(7, 5), extra=0)
+    Q = 3
+    q = rng.standard_normal((2, Q, 4, 10))
+    qpos = np.stack([c["seq_len"] - Q + i for i in range(Q)], axis=1)
+    args = dict(M=c["M"], V=c["V"], k_rope=c["k_rope"], seq_offset=c["seq_offset"],
+                seq_len=c["seq_len"], d_n=6, d_r=4, base=10000.0)
+    out, lse = orc.gva_decode_multi(q=q, q_pos=qpos, **args)
+    one, one_l = orc.gva_decode_multi(q=q[:, :1], q_pos=c["seq_len"][:, None], **args)
+    ref1, ref1_l = orc.gva_decode(q=q[:, 0], q_pos=c["seq_len"], **args)
+    assert np.array_equal(one[:, 0], ref1) and np.array_equal(one_l[:, 0], ref1_l)
+    last, last_l = orc.gva_decode(q=q[:, Q - 1], q_pos=qpos[:, Q - 1], **args)
+    assert np.max(np.abs(out[:, Q - 1] - last)) < 1e-14
+    V2 = c["V"].copy()
+    for b in range(2):                         # change the last row of every sequence
+        V2[c["seq_offset"][b] + c["seq_len"][b] - 1] += 1.0
+    out2, _ = orc.gva_decode_multi(q=q, q_pos=qpos, **dict(args, V=V2))
+    assert np.max(np.abs(out2[:, :Q - 1] - out[:, :Q - 1])) == 0
+    assert np.max(np.abs(out2[:, Q - 1] - out[:, Q - 1])) > 1e-6
+
+
 ALL_CHECKS = [check_cache_ratio, check_kv_shared_is_sdpa, check_gqa_is_sdpa, check_rope_matches_llama,
               check_relative_position, check_rope_group_law, check_absorption_identity,
-              check_softmax_closed_forms, check_bruteforce, check_round_to_bf16, check_append]
+              check_softmax_closed_forms, check_bruteforce, check_round_to_bf16, check_append,
+              check_multi_query_causal]

@@ -146,10 +146,27 @@ def _mut_append_no_rotate(m):
     m.append_cache = bad
 
 
+def _mut_causal_off_by_one(m):
+    orig = m.gva_decode
+
+    def multi(q, M, q_pos, V, k_rope, seq_offset, seq_len, d_n, d_r, base, scale=None):
+        q = np.asarray(q, dtype=float)
+        Q = q.shape[1]
+        outs, lses = [], []
+        for i in range(Q):                       # sees one row past its own position
+            Li = np.minimum(np.asarray(seq_len) - Q + i + 2, np.asarray(seq_len))
+            o, l = orig(q[:, i], M, np.asarray(q_pos)[:, i], V, k_rope, seq_offset, Li, d_n, d_r,
+                        base, scale=scale)
+            outs.append(o)
+            lses.append(l)
+        return np.stack(outs, 1), np.stack(lses, 1)
+    m.gva_decode_multi = multi
+
+
 MUTATIONS = [_mut_rope_sign, _mut_rope_adjacent_pairs, _mut_rope_freq, _mut_drop_rope_term,
              _mut_group_map, _mut_transposed_map, _mut_scale, _mut_softmax_no_norm,
              _mut_off_by_one_len, _mut_gqa_group_map, _mut_bf16_truncate, _mut_cache_count,
-             _mut_append_no_rotate]
+             _mut_append_no_rotate, _mut_causal_off_by_one]
 
 
 @pytest.mark.parametrize("mutate", MUTATIONS, ids=lambda f: f.__name__[5:])
