@@ -31,27 +31,30 @@ __global__ void __launch_bounds__(1024)
   const int tid = threadIdx.x, lane = tid & 31, pg = tid >> 5, npg = blockDim.x >> 5;
   const bool scan = a.B <= kCombineScanMaxB;
   if (scan && pg == 0) {
-    // lengths of sequences < b, of b, and of the whole batch (one warp)
-    long long before = 0, total = 0;
-    int Lb = 0;
+    // tokens of the whole batch, tiles of sequences < b, of b and of the batch
+    // (one warp), then the CTAs that own the first and last tile of b
+    long long total = 0, before = 0, tiles = 0;
+    int nb = 0;
     for (int j = lane; j < a.B; j += 32) {
       const int L = max(__ldg(a.seq_len + j), 0);
+      const int n = (L + a.tile - 1) / a.tile;
       total += L;
-      if (j < b) before += L;
-      if (j == b) Lb = L;
+      tiles += n;
+      if (j < b) before += n;
+      if (j == b) nb = n;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      before += __shfl_xor_sync(0xffffffffu, before, o);
       total += __shfl_xor_sync(0xffffffffu, total, o);
-      Lb += __shfl_xor_sync(0xffffffffu, Lb, o);
+      before += __shfl_xor_sync(0xffffffffu, before, o);
+      tiles += __shfl_xor_sync(0xffffffffu, tiles, o);
+      nb += __shfl_xor_sync(0xffffffffu, nb, o);
     }
     if (lane == 0) {
       int first = 0, count = 0;
-      if (Lb > 0 && total < (1ll << 31)) {
-        const int per = (int)((total + a.grid - 1) / a.grid);
-        const int span = max(a.tile, (per + a.tile - 1) / a.tile * a.tile);
-        const int f = (int)(before / span), l = (int)((before + Lb - 1) / span);
+      if (nb > 0 && total < (1ll << 31)) {
+        const TileSplit ts{(int)tiles, a.grid};
+        const int f = ts.cta_of((int)before), l = ts.cta_of((int)before + nb - 1);
         first = f + b;
         count = l - f + 1;
       }

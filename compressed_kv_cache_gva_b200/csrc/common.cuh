@@ -81,20 +81,41 @@ __device__ __forceinline__ void trace_mark(const DecodeArgs& a, int slot) {
 }
 
 // ---------------------------------------------------------------------------
-// Split-KV work list.  Tokens of all sequences are concatenated in batch order;
-// CTA i owns the span [i*span, (i+1)*span) of that order with
-// span = ceil(total/grid) rounded up to `tile`.  The intersection of the span
-// with sequence b is one "piece"; it is written to partial slot i + b.  Two
+// Split-KV work list.  Sequence b is cut into nt_b = ceil(L_b / TT) tiles of TT
+// tokens (the last one ragged); the tiles of the batch are numbered in batch
+// order (tile prefix tp[b]) and CTA i owns tiles [first(i), first(i+1)) with
+// first(i) = floor(i * NT / grid).  Cutting at tile boundaries keeps every CTA at
+// ceil(NT / grid) tiles or fewer: a token-balanced cut would hand a CTA whose
+// range crosses the end of a sequence two ragged tiles.  The tiles CTA i owns in
+// sequence b form one "piece"; it is written to partial slot i + b.  Two
 // non-empty pieces (b, i) and (b', i') with b + i = b' + i' cannot exist:
-// sequences are contiguous in the concatenated order, so b' > b forces i' >= i.
+// sequences are contiguous in the tile order, so b' > b forces i' >= i.
 // ---------------------------------------------------------------------------
-__device__ inline long long block_scan_lengths(const int* __restrict__ seq_len, int B,
-                                               int* prefix, long long* warp_tmp) {
+struct TileSplit {
+  int NT;     // tiles in the batch
+  int grid;   // CTAs
+  __device__ __forceinline__ bool narrow() const { return NT <= 0x7fffffff / grid; }
+  __device__ __forceinline__ int first(int i) const {
+    return narrow() ? (int)((unsigned)(i * NT) / (unsigned)grid)
+                    : (int)((long long)i * NT / grid);
+  }
+  // the CTA that owns tile u (0 <= u < NT): the last i with first(i) <= u
+  __device__ __forceinline__ int cta_of(int u) const {
+    return narrow() ? (int)((unsigned)((u + 1) * grid - 1) / (unsigned)NT)
+                    : (int)(((long long)(u + 1) * grid - 1) / NT);
+  }
+};
+
+// Exclusive prefix sums of val(0..B-1) (each >= 0) into prefix[0..B], for the
+// whole block; returns the total.  If the total does not fit in int, every
+// entry is 0 (the caller flags it).
+template <class F>
+__device__ inline long long block_scan(int B, F val, int* prefix, long long* warp_tmp) {
   const int tid = threadIdx.x, nt = blockDim.x;
   const int per = (B + nt - 1) / nt;
   const int beg = min(tid * per, B), end = min(beg + per, B);
   long long sum = 0;
-  for (int b = beg; b < end; ++b) sum += max(__ldg(seq_len + b), 0);
+  for (int b = beg; b < end; ++b) sum += val(b);
   const int lane = tid & 31, w = tid >> 5;
   long long incl = sum;
 #pragma unroll
@@ -122,27 +143,75 @@ __device__ inline long long block_scan_lengths(const int* __restrict__ seq_len, 
   const bool fits = total < (1ll << 31);
   for (int b = beg; b < end; ++b) {
     prefix[b] = fits ? (int)run : 0;
-    run += max(__ldg(seq_len + b), 0);
+    run += val(b);
   }
   if (tid == 0) prefix[B] = fits ? (int)total : 0;
-  __syncthreads();
+  __syncthreads();   // prefix complete; warp_tmp free again
   return total;
 }
 
-struct Span {
-  int span;    // tokens per CTA
-  int total;   // tokens in the batch
-};
-
-__device__ inline Span make_span(int total, int grid, int tile) {
-  Span s;
-  s.total = total;
-  int per = (total + grid - 1) / grid;
-  s.span = max(tile, (per + tile - 1) / tile * tile);
-  return s;
+// Token prefix of the lengths (negative lengths count as 0).
+__device__ inline long long block_scan_lengths(const int* __restrict__ seq_len, int B,
+                                               int* prefix, long long* warp_tmp) {
+  return block_scan(B, [&](int b) { return (long long)max(__ldg(seq_len + b), 0); }, prefix,
+                    warp_tmp);
 }
 
-// First sequence whose token range ends after `pos` (skips empty sequences).
+// Tile prefix tp[] from the token prefix, tiles of tt tokens.
+__device__ inline int block_scan_tiles(const int* prefix, int B, int tt, int* tp,
+                                       long long* warp_tmp) {
+  return (int)block_scan(
+      B, [&](int b) { return (long long)((prefix[b + 1] - prefix[b] + tt - 1) / tt); }, tp,
+      warp_tmp);
+}
+
+// Token prefix prefix[0..B] and tile prefix tp[0..B] (tiles of TT tokens) of the
+// batch for the whole block; returns the token total (every entry is 0 when the
+// total exceeds 2^31 - 1, which the caller flags).  For B <= 32 one warp scans
+// the lengths its lanes already loaded (len_lane: the lane's length, 0 for lanes
+// >= B), with no block-wide scan; larger batches take two block scans.
+template <int TT>
+__device__ inline long long scan_batch(const int* __restrict__ seq_len, int B, int len_lane,
+                                       int* prefix, int* tp, long long* warp_tmp) {
+  if (B > 32) {
+    const long long total = block_scan_lengths(seq_len, B, prefix, warp_tmp);
+    block_scan_tiles(prefix, B, TT, tp, warp_tmp);
+    return total;
+  }
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int L = max(len_lane, 0);
+    const unsigned n = (unsigned)(L + TT - 1) / TT;
+    long long x = L;
+    unsigned y = n;          // tiles never exceed tokens, so they fit whenever the total does
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long u = __shfl_up_sync(0xffffffffu, x, o);
+      const unsigned v = __shfl_up_sync(0xffffffffu, y, o);
+      if (lane >= o) {
+        x += u;
+        y += v;
+      }
+    }
+    const long long total = __shfl_sync(0xffffffffu, x, 31);
+    const unsigned tiles = __shfl_sync(0xffffffffu, y, 31);
+    const bool fits = total < (1ll << 31);
+    if (lane < B) {
+      prefix[lane] = fits ? (int)(x - L) : 0;
+      tp[lane] = fits ? (int)(y - n) : 0;
+    }
+    if (lane == 0) {
+      prefix[B] = fits ? (int)total : 0;
+      tp[B] = fits ? (int)tiles : 0;
+      warp_tmp[32] = total;
+    }
+  }
+  __syncthreads();
+  return warp_tmp[32];
+}
+
+// First sequence whose range in a prefix array ends after `pos` (skips empty
+// sequences).
 __device__ inline int seq_at(const int* prefix, int B, int pos) {
   int lo = 0, hi = B;  // answer in [0, B]
   while (lo < hi) {
@@ -152,35 +221,53 @@ __device__ inline int seq_at(const int* prefix, int B, int pos) {
   return lo;
 }
 
-// Walks the tiles of one CTA's span: sequence b, tile start t0 (token index in the
+// The tile range [T0, T1) of one CTA and its pieces.
+struct CtaTiles {
+  const int* prefix;   // token prefix [B+1]
+  const int* tp;       // tile prefix [B+1]
+  int B, T0, T1, tt;
+  __device__ __forceinline__ bool empty() const { return T1 <= T0; }
+  __device__ __forceinline__ int first_seq() const { return empty() ? B : seq_at(tp, B, T0); }
+  // does sequence b start before this CTA's range ends?
+  __device__ __forceinline__ bool reaches(int b) const { return b < B && tp[b] < T1; }
+  // token range [j0, j1) of sequence b inside this CTA's tiles; false if empty
+  __device__ __forceinline__ bool piece(int b, int& j0, int& j1) const {
+    const int u0 = max(T0, tp[b]) - tp[b], u1 = min(T1, tp[b + 1]) - tp[b];
+    j0 = u0 * tt;
+    j1 = min(u1 * tt, prefix[b + 1] - prefix[b]);
+    return j1 > j0;
+  }
+};
+
+// Walks the tiles of one CTA: sequence b, tile start t0 (token index in the
 // sequence) and the piece end j1.  Empty sequences are skipped; b == B means done.
 struct TileCursor {
   int b, t0, j1;
-  __device__ void seek(const int* prefix, int B, int s0, int s1, int from) {
-    for (b = from; b < B && prefix[b] < s1; ++b) {
-      const int j0 = max(s0, prefix[b]) - prefix[b];
-      j1 = min(s1, prefix[b + 1]) - prefix[b];
-      if (j1 > j0) {
+  __device__ void seek(const CtaTiles& r, int from) {
+    for (b = from; r.reaches(b); ++b) {
+      int j0;
+      if (r.piece(b, j0, j1)) {
         t0 = j0;
         return;
       }
     }
-    b = B;
+    b = r.B;
   }
-  __device__ void next(const int* prefix, int B, int s0, int s1, int tile) {
-    t0 += tile;
-    if (t0 >= j1) seek(prefix, B, s0, s1, b + 1);
+  __device__ void next(const CtaTiles& r) {
+    t0 += r.tt;
+    if (t0 >= j1) seek(r, b + 1);
   }
 };
 
 // CTA 0 records, for every sequence, where its pieces land and how many there are,
 // and flags sequences whose slots leave the cache.
-__device__ inline void write_meta(const DecodeArgs& a, const int* prefix, Span sp) {
+__device__ inline void write_meta(const DecodeArgs& a, const int* prefix, const int* tp,
+                                  TileSplit ts) {
   for (int b = threadIdx.x; b < a.B; b += blockDim.x) {
     int L = prefix[b + 1] - prefix[b];
     int2 m = make_int2(0, 0);
     if (L > 0) {
-      int first = prefix[b] / sp.span, last = (prefix[b + 1] - 1) / sp.span;
+      const int first = ts.cta_of(tp[b]), last = ts.cta_of(tp[b + 1] - 1);
       m = make_int2(first + b, last - first + 1);
       long long off = __ldg(a.seq_offset + b);
       if (off < 0 || off + L > a.num_slots) atomicOr(a.status, GVA_DEVERR_RANGE);

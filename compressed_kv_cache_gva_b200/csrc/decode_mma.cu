@@ -58,14 +58,15 @@ int mma_tile(const gva_shape_t& sh, bool gqa) {
 }
 
 int mma_grid(const gva_shape_t& sh, int num_sms, long long max_total_tokens, bool gqa) {
-  int tt = 16;
+  int tt = 16, minb = 2;
   size_t smem = 0;
   dispatch(sh, gqa, [&](auto c) {
     tt = decltype(c)::TT;
+    minb = decltype(c)::MINB;
     smem = decltype(c)::smem_bytes(sh.B);
   });
   int per_sm = (int)((227 * 1024) / (smem + 1024));
-  per_sm = per_sm < 1 ? 1 : (per_sm > 2 ? 2 : per_sm);
+  per_sm = per_sm < 1 ? 1 : (per_sm > minb ? minb : per_sm);
   if (sh.ctas_per_sm > 0) per_sm = sh.ctas_per_sm;
   long long want = (max_total_tokens + tt - 1) / tt;
   long long grid = (long long)num_sms * per_sm;

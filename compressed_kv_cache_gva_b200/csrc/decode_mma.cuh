@@ -67,22 +67,27 @@ struct MmaCfg {
   // end-of-piece merge of the W warps of a group: (m, l) per warp and lane quad,
   // and the output fragments of warps 1..W-1
   static constexpr int MERGE_ML = W * 4 * 4;                    // floats per group
-  static constexpr int MERGE_O = (W - 1) * 32 * NT * KS * 4;   // floats per group
+  static constexpr int MERGE_O = (W - 1) * 32 * KS * 4;        // floats per group
   static constexpr int MERGE = W > 1 ? NG * (MERGE_ML + MERGE_O) * 4 : 0;  // bytes
   static constexpr int KR_SW = DRP * 2;               // swizzle span of the k_rope box
+  // resident CTAs per SM the register budget is sized for.  Two CTAs of 9 warps
+  // leave 96 registers a thread; 8 columns of d_h = 128 keep ~100 values live in
+  // the consumer (query fragments, O^T accumulators, V^T fragments), so that
+  // configuration runs one CTA per SM instead of spilling.
+  static constexpr int MINB = (NCW >= 8 && HPG == 8 && D_H == 128) ? 1 : 2;
   static_assert(HPG == 4 || HPG == 8, "heads per group");
   static_assert(STAGES % W == 0, "each stage must belong to one warp of a group");
   static_assert(D_H % 64 == 0, "d_h");
   static_assert(DRP == 0 || DRP == 16 || DRP == 32, "padded d_r");
 
   static size_t smem_bytes(int B) {
-    return 1024 + PIPE + MERGE + 16 * STAGES + 2 * sizeof(int) * (B + 1) + 16 +
+    return 1024 + PIPE + MERGE + 16 * STAGES + 3 * sizeof(int) * (B + 1) + 16 +
            sizeof(long long) * 33;
   }
 };
 
 template <class C>
-__global__ void __launch_bounds__(C::THREADS, 2)
+__global__ void __launch_bounds__(C::THREADS, C::MINB)
     decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_x,
                       const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_kr) {
@@ -94,9 +99,19 @@ __global__ void __launch_bounds__(C::THREADS, 2)
   uint64_t* empty = full + C::STAGES;
   int* prefix = reinterpret_cast<int*>(empty + C::STAGES);
   int* offs = prefix + a.B + 1;
+  int* tp = offs + a.B + 1;            // tile prefix
   long long* wtmp = reinterpret_cast<long long*>(
-      (reinterpret_cast<uintptr_t>(offs + a.B + 1) + 15) & ~uintptr_t(15));
+      (reinterpret_cast<uintptr_t>(tp + a.B + 1) + 15) & ~uintptr_t(15));
 
+  // The lengths and offsets are caller inputs that no kernel of this library
+  // writes: they are requested first, so that their latency overlaps the barrier
+  // setup, and read before waiting on the preceding kernel.
+  const bool small_b = a.B <= 32;
+  int len_lane = 0, off_lane = 0;
+  if (small_b && threadIdx.x < a.B) {
+    len_lane = __ldg(a.seq_len + threadIdx.x);
+    off_lane = __ldg(a.seq_offset + threadIdx.x);
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) trace_mark(a, 0);
   if (threadIdx.x == 0) {
@@ -111,20 +126,19 @@ __global__ void __launch_bounds__(C::THREADS, 2)
     if (C::GQA) prefetch_tmap(&tm_v);
     if (C::DRP) prefetch_tmap(&tm_kr);
   }
-  // The lengths and offsets are caller inputs that no kernel of this library
-  // writes, so they are read before waiting on the preceding kernel.
-  for (int b = threadIdx.x; b < a.B; b += blockDim.x) offs[b] = __ldg(a.seq_offset + b);
-  long long total64 = block_scan_lengths(a.seq_len, a.B, prefix, wtmp);   // syncs the block
-  int total = (int)total64;
-  if (total64 >= (1ll << 31)) {
-    if (threadIdx.x == 0) atomicOr(a.status, GVA_DEVERR_RANGE);
-    total = 0;
+  if (small_b) {
+    if (threadIdx.x < a.B) offs[threadIdx.x] = off_lane;
+  } else {
+    for (int b = threadIdx.x; b < a.B; b += blockDim.x) offs[b] = __ldg(a.seq_offset + b);
   }
-  const Span sp = make_span(total, gridDim.x, C::TT);
-  const int s0 = blockIdx.x * sp.span;
-  const bool has_work = s0 < total;
-  const int s1 = min(s0 + sp.span, total);
-  const int b_first = has_work ? seq_at(prefix, a.B, s0) : a.B;
+  // token and tile prefixes (all zeros, and flagged, past 2^31 - 1 tokens)
+  if (scan_batch<C::TT>(a.seq_len, a.B, len_lane, prefix, tp, wtmp) >= (1ll << 31) &&
+      threadIdx.x == 0)
+    atomicOr(a.status, GVA_DEVERR_RANGE);
+  const TileSplit ts{tp[a.B], (int)gridDim.x};
+  const CtaTiles rng{prefix, tp, a.B, ts.first(blockIdx.x), ts.first(blockIdx.x + 1), C::TT};
+  const bool has_work = !rng.empty();
+  const int b_first = rng.first_seq();
 
   // ------------------------------------------------------------------ producer
   // One thread issues every load of the CTA.  The cache is read once per step:
@@ -171,9 +185,9 @@ __global__ void __launch_bounds__(C::THREADS, 2)
       for (int i = threadIdx.x; i < a.n_new; i += blockDim.x) {
         const long long sl = __ldg(a.new_slots + i);
         int kbase = 0;
-        for (int b = b_first; b < a.B && prefix[b] < s1; ++b) {
-          const int j0 = max(s0, prefix[b]) - prefix[b], j1 = min(s1, prefix[b + 1]) - prefix[b];
-          if (j1 <= j0) continue;
+        for (int b = b_first; rng.reaches(b); ++b) {
+          int j0, j1;
+          if (!rng.piece(b, j0, j1)) continue;
           const long long r0 = (long long)offs[b] + j0, r1 = (long long)offs[b] + j1;
           if (sl >= r0 && sl < r1) atomicMin(&first_dirty, kbase + (int)((sl - r0) / C::TT));
           kbase += (j1 - j0 + C::TT - 1) / C::TT;
@@ -183,19 +197,19 @@ __global__ void __launch_bounds__(C::THREADS, 2)
   }
   if (producer) {
     pol = policy_evict_first();
-    cur.seek(prefix, a.B, s0, s1, b_first);
+    cur.seek(rng, b_first);
     if (a.prefetch) {
       const int limit = min(C::STAGES, first_dirty);
       for (; cur.b < a.B && k_issued < limit; ++k_issued) {
         issue(k_issued);
-        cur.next(prefix, a.B, s0, s1, C::TT);
+        cur.next(rng);
       }
     }
   }
   pdl_wait();
   pdl_trigger();
   if (threadIdx.x == 0) trace_mark(a, 1);
-  if (blockIdx.x == 0) write_meta(a, prefix, sp);
+  if (blockIdx.x == 0) write_meta(a, prefix, tp, ts);
   if (!has_work) return;
 
   if (warp == C::NCW) {
@@ -209,7 +223,7 @@ __global__ void __launch_bounds__(C::THREADS, 2)
         break;
       }
       issue(k);
-      cur.next(prefix, a.B, s0, s1, C::TT);
+      cur.next(rng);
     }
     (void)prod_ok;
     // Drain: do not leave while a copy into this CTA's shared memory is in flight.
@@ -244,9 +258,9 @@ __global__ void __launch_bounds__(C::THREADS, 2)
   bool ok = true;   // false once a bounded wait gave up: skip work, keep barrier order
 
   int k = 0;
-  for (int b = b_first; b < a.B && prefix[b] < s1; ++b) {
-    const int j0 = max(s0, prefix[b]) - prefix[b], j1 = min(s1, prefix[b + 1]) - prefix[b];
-    if (j1 <= j0) continue;
+  for (int b = b_first; rng.reaches(b); ++b) {
+    int j0, j1;
+    if (!rng.piece(b, j0, j1)) continue;
 
     // ---- query fragments (B operand of the score MMA): column n = gq
     uint32_t qb[C::NT][C::KS][2];
@@ -306,13 +320,14 @@ __global__ void __launch_bounds__(C::THREADS, 2)
       }
     }
 
-    float o[C::NT][C::KS][4];
+    // O^T fragments: d rows x 8 columns.  With 8 columns per group the hi and lo
+    // halves of P (two n-tiles) belong to the same heads and share these
+    // accumulators; with 4 the lo half sits in the upper 4 columns (merged at the end)
+    float o[C::KS][4];
 #pragma unroll
-    for (int nt = 0; nt < C::NT; ++nt)
+    for (int md = 0; md < C::KS; ++md)
 #pragma unroll
-      for (int md = 0; md < C::KS; ++md)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[nt][md][e] = 0.f;
+      for (int e = 0; e < 4; ++e) o[md][e] = 0.f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     // causal limits of this thread's two columns: the nq new tokens sit at
     // positions L-nq .. L-1 and query i sees the cache up to its own position
@@ -444,23 +459,21 @@ __global__ void __launch_bounds__(C::THREADS, 2)
       l0 = l0 * al0 + rs0;
       l1 = l1 * al1 + rs1;
 #pragma unroll
-      for (int nt = 0; nt < C::NT; ++nt)
-#pragma unroll
-        for (int md = 0; md < C::KS; ++md) {
-          o[nt][md][0] *= al0;
-          o[nt][md][1] *= al1;
-          o[nt][md][2] *= al0;
-          o[nt][md][3] *= al1;
-        }
+      for (int md = 0; md < C::KS; ++md) {
+        o[md][0] *= al0;
+        o[md][1] *= al1;
+        o[md][2] *= al0;
+        o[md][3] *= al1;
+      }
 
       // ---- O^T += V^T P over this warp's tokens (V^T fragments loaded above)
 #pragma unroll
       for (int mm = 0; mm < C::MW; ++mm)
 #pragma unroll
-        for (int md = 0; md < C::KS; ++md)
+        for (int nt = 0; nt < C::NT; ++nt)
 #pragma unroll
-          for (int nt = 0; nt < C::NT; ++nt)
-            mma_bf16(o[nt][md], vf[mm][md][0], vf[mm][md][1], vf[mm][md][2], vf[mm][md][3],
+          for (int md = 0; md < C::KS; ++md)
+            mma_bf16(o[md], vf[mm][md][0], vf[mm][md][1], vf[mm][md][2], vf[mm][md][3],
                      bp[mm][nt][0], bp[mm][nt][1]);
       if (ragged) fence_proxy_async_smem();
       __syncwarp();
@@ -504,51 +517,44 @@ __global__ void __launch_bounds__(C::THREADS, 2)
       }
       const float f0 = ex2(m0 - Ms0), f1 = ex2(m1 - Ms1);
 #pragma unroll
-      for (int nt = 0; nt < C::NT; ++nt)
-#pragma unroll
-        for (int md = 0; md < C::KS; ++md) {
-          o[nt][md][0] *= f0;
-          o[nt][md][1] *= f1;
-          o[nt][md][2] *= f0;
-          o[nt][md][3] *= f1;
-        }
+      for (int md = 0; md < C::KS; ++md) {
+        o[md][0] *= f0;
+        o[md][1] *= f1;
+        o[md][2] *= f0;
+        o[md][3] *= f1;
+      }
       m0 = M0; m1 = M1; l0 = L0; l1 = L1;
       if (w > 0) {
-        float* dst = mg_o + ((w - 1) * 32 + lane) * (C::NT * C::KS * 4);
+        float* dst = mg_o + ((w - 1) * 32 + lane) * (C::KS * 4);
 #pragma unroll
-        for (int nt = 0; nt < C::NT; ++nt)
-#pragma unroll
-          for (int md = 0; md < C::KS; ++md)
-            *reinterpret_cast<float4*>(dst + (nt * C::KS + md) * 4) =
-                make_float4(o[nt][md][0], o[nt][md][1], o[nt][md][2], o[nt][md][3]);
+        for (int md = 0; md < C::KS; ++md)
+          *reinterpret_cast<float4*>(dst + md * 4) =
+              make_float4(o[md][0], o[md][1], o[md][2], o[md][3]);
       }
       named_bar_sync(bar, nthr);
       if (w == 0) {
 #pragma unroll
         for (int u = 1; u < C::W; ++u) {
-          const float* src = mg_o + ((u - 1) * 32 + lane) * (C::NT * C::KS * 4);
+          const float* src = mg_o + ((u - 1) * 32 + lane) * (C::KS * 4);
 #pragma unroll
-          for (int nt = 0; nt < C::NT; ++nt)
-#pragma unroll
-            for (int md = 0; md < C::KS; ++md) {
-              const float4 x = *reinterpret_cast<const float4*>(src + (nt * C::KS + md) * 4);
-              o[nt][md][0] += x.x;
-              o[nt][md][1] += x.y;
-              o[nt][md][2] += x.z;
-              o[nt][md][3] += x.w;
-            }
+          for (int md = 0; md < C::KS; ++md) {
+            const float4 x = *reinterpret_cast<const float4*>(src + md * 4);
+            o[md][0] += x.x;
+            o[md][1] += x.y;
+            o[md][2] += x.z;
+            o[md][3] += x.w;
+          }
         }
       }
       named_bar_sync(bar, nthr);   // scratch free for the next piece
     }
     if (w != 0) continue;
+    if constexpr (C::HPG == 4) {
 #pragma unroll
-    for (int md = 0; md < C::KS; ++md)
+      for (int md = 0; md < C::KS; ++md)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if constexpr (C::HPG == 8) o[0][md][e] += o[1][md][e];
-        else o[0][md][e] += __shfl_xor_sync(0xffffffffu, o[0][md][e], 2);
-      }
+        for (int e = 0; e < 4; ++e) o[md][e] += __shfl_xor_sync(0xffffffffu, o[md][e], 2);
+    }
     if (ok && (C::HPG == 8 || t < 2)) {
       const size_t slot = (size_t)blockIdx.x + b;
       float* po0 = a.part_o + (slot * Hp + phead0) * C::D_H;
@@ -556,10 +562,10 @@ __global__ void __launch_bounds__(C::THREADS, 2)
 #pragma unroll
       for (int md = 0; md < C::KS; ++md) {
         const int d = md * 16 + gq;
-        po0[d] = o[0][md][0];
-        po1[d] = o[0][md][1];
-        po0[d + 8] = o[0][md][2];
-        po1[d + 8] = o[0][md][3];
+        po0[d] = o[md][0];
+        po1[d] = o[md][1];
+        po0[d + 8] = o[md][2];
+        po1[d + 8] = o[md][3];
       }
       if (gq == 0) {
         a.part_ml[slot * Hp + phead0] = make_float2(m0, l0);

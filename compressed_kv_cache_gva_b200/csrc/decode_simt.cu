@@ -21,7 +21,7 @@ constexpr int kSimtOPT = 16;   // outputs per thread: H*d_h <= 4096
 
 struct SimtLayout {
   int row;           // elements per cache row (G*d_h)
-  size_t xs, vs, krs, qs, ss, mrun, lrun, alpha, prefix, wtmp, total;
+  size_t xs, vs, krs, qs, ss, mrun, lrun, alpha, prefix, tp, wtmp, total;
 };
 
 static SimtLayout simt_layout(const gva_shape_t& sh, bool gqa) {
@@ -39,6 +39,7 @@ static SimtLayout simt_layout(const gva_shape_t& sh, bool gqa) {
   L.lrun = take(sizeof(float) * sh.H);
   L.alpha = take(sizeof(float) * sh.H);
   L.prefix = take(sizeof(int) * (sh.B + 1));
+  L.tp = take(sizeof(int) * (sh.B + 1));
   L.wtmp = take(sizeof(long long) * 33);
   L.total = o;
   return L;
@@ -57,6 +58,7 @@ __global__ void __launch_bounds__(kSimtThreads)
   float* lrun = reinterpret_cast<float*>(sm + Ly.lrun);
   float* alpha = reinterpret_cast<float*>(sm + Ly.alpha);
   int* prefix = reinterpret_cast<int*>(sm + Ly.prefix);
+  int* tp = reinterpret_cast<int*>(sm + Ly.tp);
   long long* wtmp = reinterpret_cast<long long*>(sm + Ly.wtmp);
 
   const int H = a.H, d_h = a.d_h, hpg = a.H / a.G, row = Ly.row;
@@ -69,21 +71,17 @@ __global__ void __launch_bounds__(kSimtThreads)
 
   pdl_wait();
   pdl_trigger();
-  long long total64 = block_scan_lengths(a.seq_len, a.B, prefix, wtmp);
-  int total = (int)total64;
-  if (total64 >= (1ll << 31)) {
-    if (tid == 0) atomicOr(a.status, GVA_DEVERR_RANGE);
-    total = 0;
-  }
-  const Span sp = make_span(total, gridDim.x, kSimtTT);
-  if (blockIdx.x == 0) write_meta(a, prefix, sp);
-  const int s0 = blockIdx.x * sp.span;
-  if (s0 >= total) return;
-  const int s1 = min(s0 + sp.span, total);
+  const int len_lane = (a.B <= 32 && tid < a.B) ? __ldg(a.seq_len + tid) : 0;
+  if (scan_batch<kSimtTT>(a.seq_len, a.B, len_lane, prefix, tp, wtmp) >= (1ll << 31) && tid == 0)
+    atomicOr(a.status, GVA_DEVERR_RANGE);
+  const TileSplit ts{tp[a.B], (int)gridDim.x};
+  if (blockIdx.x == 0) write_meta(a, prefix, tp, ts);
+  const CtaTiles rng{prefix, tp, a.B, ts.first(blockIdx.x), ts.first(blockIdx.x + 1), kSimtTT};
+  if (rng.empty()) return;
 
-  for (int b = seq_at(prefix, a.B, s0); b < a.B && prefix[b] < s1; ++b) {
-    const int j0 = max(s0, prefix[b]) - prefix[b], j1 = min(s1, prefix[b + 1]) - prefix[b];
-    if (j1 <= j0) continue;
+  for (int b = rng.first_seq(); rng.reaches(b); ++b) {
+    int j0, j1;
+    if (!rng.piece(b, j0, j1)) continue;
     const long long row0 = __ldg(a.seq_offset + b);
     // query of sequence b, base-2 scaled
     for (int e = tid; e < H * dq; e += blockDim.x) {
