@@ -410,7 +410,7 @@ def run_ours(args, rank, world, local):
                    "parallelism": (f"sequence split: each sequence's cache over {world} GPU(s), "
                                    "NCCL all-gather of (out, lse) + merge") if split_seq else
                                   f"weak: {world} independent batch(es), one per GPU",
-                   "step": "gva_decode_step: append + absorb + decode (split + combine)",
+                   "step": "gva_decode_step: append + absorb (one kernel), decode (split + combine)",
                    "graphs": "CUDA graphs",
                    "decode_path": "fma" if args.fma else "tensor"},
         "steps_per_s": round(world * K / (ms * 1e-3), 1),
@@ -435,7 +435,7 @@ def run_ours(args, rank, world, local):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(ms_e2e / K, 6)},
         "multi_token": multi,
-        "gpu_launches": (5 if split_seq else 4) * K,
+        "gpu_launches": (4 if split_seq else 3) * K,
         "clocks": clocks,
     }
     return res, di

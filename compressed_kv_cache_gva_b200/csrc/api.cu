@@ -259,18 +259,40 @@ const char* gva_last_error(void) { return g_err; }
 void gva_trace_set_buffer(void* dev_buf) { g_trace = static_cast<unsigned long long*>(dev_buf); }
 #endif
 
-static gva_status_t absorb_impl(const gva_shape_t* shp, const void* q, const void* M,
-                                const int32_t* q_pos, float* q_abs, void* stream, bool early) {
-  gva_status_t s = check_shape(shp, false);
-  if (s != GVA_OK) return s;
-  const gva_shape_t& sh = *shp;
-  if (sh.B == 0) return GVA_OK;
+// Argument checks of the absorb (shape already checked; B > 0).
+static gva_status_t absorb_check(const gva_shape_t& sh, const void* q, const void* M,
+                                 const int32_t* q_pos, const float* q_abs) {
   if (!q || !q_abs || !q_pos || (sh.d_n > 0 && !M))
     return fail(GVA_ERR_INVALID_ARG, "a required pointer is NULL");
   if (!aligned16(q) || (M && !aligned16(M)) || !aligned16(q_pos) || !aligned16(q_abs))
     return fail(GVA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   const size_t smem = gva::absorb_smem_bytes(sh);
   if (smem > 200 * 1024) return fail(GVA_ERR_UNSUPPORTED, "M_h too large for one CTA (%zu bytes)", smem);
+  return GVA_OK;
+}
+
+// Argument checks of the append (shape already checked; N > 0).
+static gva_status_t append_check(const gva_shape_t& sh, const void* v_new, const void* kpe_new,
+                                 const int32_t* slot, const int32_t* pos, int64_t num_slots,
+                                 const void* V_cache, const void* kr_cache) {
+  if (!v_new || !slot || !pos || !V_cache || (sh.d_r > 0 && (!kpe_new || !kr_cache)))
+    return fail(GVA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned16(v_new) || !aligned16(V_cache) || (kpe_new && !aligned16(kpe_new)) ||
+      (kr_cache && !aligned16(kr_cache)) || !aligned16(slot) || !aligned16(pos))
+    return fail(GVA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if ((sh.G * sh.d_h * elt(sh.cache_dtype)) % 16)
+    return fail(GVA_ERR_INVALID_ARG, "value rows must be multiples of 16 bytes");
+  if (num_slots < 1) return fail(GVA_ERR_INVALID_ARG, "num_slots=%lld < 1", (long long)num_slots);
+  return GVA_OK;
+}
+
+static gva_status_t absorb_impl(const gva_shape_t* shp, const void* q, const void* M,
+                                const int32_t* q_pos, float* q_abs, void* stream, bool early) {
+  gva_status_t s = check_shape(shp, false);
+  if (s != GVA_OK) return s;
+  const gva_shape_t& sh = *shp;
+  if (sh.B == 0) return GVA_OK;
+  if ((s = absorb_check(sh, q, M, q_pos, q_abs)) != GVA_OK) return s;
   const float c = scale_of(sh, false) * gva::kLog2e;
   cudaError_t e =
       gva::launch_absorb(sh, q, M, q_pos, q_abs, c, static_cast<cudaStream_t>(stream), early);
@@ -286,14 +308,8 @@ static gva_status_t append_impl(const gva_shape_t* shp, int32_t N, const void* v
   const gva_shape_t& sh = *shp;
   if (N < 0) return fail(GVA_ERR_INVALID_ARG, "N=%d < 0", N);
   if (N == 0) return GVA_OK;
-  if (!v_new || !slot || !pos || !V_cache || (sh.d_r > 0 && (!kpe_new || !kr_cache)))
-    return fail(GVA_ERR_INVALID_ARG, "a required pointer is NULL");
-  if (!aligned16(v_new) || !aligned16(V_cache) || (kpe_new && !aligned16(kpe_new)) ||
-      (kr_cache && !aligned16(kr_cache)) || !aligned16(slot) || !aligned16(pos))
-    return fail(GVA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
-  if ((sh.G * sh.d_h * elt(sh.cache_dtype)) % 16)
-    return fail(GVA_ERR_INVALID_ARG, "value rows must be multiples of 16 bytes");
-  if (num_slots < 1) return fail(GVA_ERR_INVALID_ARG, "num_slots=%lld < 1", (long long)num_slots);
+  if ((s = append_check(sh, v_new, kpe_new, slot, pos, num_slots, V_cache, kr_cache)) != GVA_OK)
+    return s;
   cudaError_t e = gva::launch_append(sh, N, v_new, kpe_new, slot, pos, num_slots, V_cache, kr_cache,
                                      err_flag, static_cast<cudaStream_t>(stream), early);
   return e == cudaSuccess ? GVA_OK : cuda_fail(e, "append launch");
@@ -351,17 +367,25 @@ gva_status_t gva_decode_step(const gva_shape_t* shape, const void* q, const void
   if ((s = plan_decode(*shape, false, max_total_tokens, &p)) != GVA_OK) return s;
   if (ws_bytes < p.ws.total)
     return fail(GVA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, p.ws.total);
-  // 1. new tokens into the cache, 2. absorbed queries, 3. decode.  This order lets
-  // the decode's split kernel start streaming the cache before it waits on the
-  // absorb kernel: absorb only triggers its successor after the append finished.
-  // Append and absorb let their successor launch immediately; every kernel still
-  // waits on its predecessor before its first store, so the chain stays ordered,
-  // and the split kernel streams all cache tiles without a new slot before it
-  // waits (its wait covers the absorb, which waited on the append).
-  if ((s = append_impl(shape, n_new, v_new, kpe_new, slot, pos, num_slots, V_cache, kr_cache,
-                       err_flag, stream, true)) != GVA_OK)
+  // 1. new tokens into the cache and absorbed queries (one kernel), 2. decode.
+  // The first kernel lets the split kernel launch immediately and waits on the
+  // preceding kernel before its first store; the split kernel streams every cache
+  // tile without a new slot before it waits on the first kernel, so the cache
+  // streams while the queries are absorbed.  Two launches instead of three save
+  // one grid-completion wait on the step's critical path.
+  if (n_new < 0) return fail(GVA_ERR_INVALID_ARG, "n_new=%d < 0", n_new);
+  if (shape->B > 0 && (s = absorb_check(*shape, q, M, q_pos, q_abs)) != GVA_OK) return s;
+  if (n_new > 0 &&
+      (s = append_check(*shape, v_new, kpe_new, slot, pos, num_slots, V_cache, kr_cache)) != GVA_OK)
     return s;
-  if ((s = absorb_impl(shape, q, M, q_pos, q_abs, stream, true)) != GVA_OK) return s;
+  {
+    const float c = scale_of(*shape, false) * gva::kLog2e;
+    cudaError_t e = gva::launch_prep_step(*shape, q, M, q_pos, q_abs, c, n_new, v_new, kpe_new,
+                                          slot, pos, num_slots, V_cache, kr_cache, err_flag,
+                                          static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "append + absorb launch");
+  }
+  if (shape->B == 0) return GVA_OK;
   return decode_common(shape, false, q_abs, V_cache, V_cache, kr_cache, seq_offset, seq_len,
                        max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream,
                        /*prefetch=*/true, slot, n_new);

@@ -80,6 +80,23 @@ __device__ __forceinline__ void trace_mark(const DecodeArgs& a, int slot) {
 #endif
 }
 
+// Per-tile timeline (same build flag): for the first 8 tiles of each CTA of the
+// split kernel, trace[65536 + (cta * 8 + k) * 4 + which] holds %globaltimer when
+// tile k was requested (which = 0), ready for group 0 (1) and released by it (2).
+__device__ __forceinline__ void trace_tile(const DecodeArgs& a, int k, int which) {
+#ifdef GVA_TRACE
+  if (a.trace && k < 8) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    a.trace[65536 + (blockIdx.x * 8 + k) * 4 + which] = t;
+  }
+#else
+  (void)a;
+  (void)k;
+  (void)which;
+#endif
+}
+
 // ---------------------------------------------------------------------------
 // Split-KV work list.  Sequence b is cut into nt_b = ceil(L_b / TT) tiles of TT
 // tokens (the last one ragged); the tiles of the batch are numbered in batch

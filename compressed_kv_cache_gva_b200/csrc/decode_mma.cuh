@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
     const int s = k % C::STAGES;
     const uint32_t fb = smem_u32(full + s);
     if (k == 0) trace_mark(a, 2);
+    trace_tile(a, k, 0);
     mbar_arrive_expect_tx(fb, C::TX);
     const uint32_t st = smem_u32(pipe + s * C::STAGE);
     const int y = offs[cur.b] + cur.t0;
@@ -347,6 +348,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       if (warp == 0 && lane == 0 && a.trace) a.trace[blockIdx.x * 8 + 6] += (unsigned long long)(tw1 - tw0);
 #endif
       if (warp == 0 && lane == 0 && k == 0) trace_mark(a, 3);
+      if (warp == 0 && lane == 0) trace_tile(a, k, 1);
       const int nvalid = min(C::TT, j1 - t0);
       uint8_t* st = pipe + s * C::STAGE;
       uint8_t* xg = st + g * C::CB * C::BOX;
@@ -478,6 +480,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       if (ragged) fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(empty + s));
+      if (warp == 0 && lane == 0) trace_tile(a, k, 2);
 #ifdef GVA_TRACE
       if (warp == 0 && lane == 0 && a.trace)
         a.trace[blockIdx.x * 8 + 7] += (unsigned long long)(clock64() - tw1);

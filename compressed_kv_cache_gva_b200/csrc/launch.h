@@ -44,6 +44,13 @@ cudaError_t launch_append(const gva_shape_t& sh, int N, const void* v_new, const
                           void* kr_cache, int* err_flag, cudaStream_t st,
                           bool early_trigger = false);
 
+// Append and absorb of the fused decode step in one launch; it lets the next
+// kernel launch at once.
+cudaError_t launch_prep_step(const gva_shape_t& sh, const void* q, const void* M, const int* q_pos,
+                             float* q_abs, float c, int N, const void* v_new, const void* kpe_new,
+                             const int* slot, const int* pos, long long num_slots, void* V_cache,
+                             void* kr_cache, int* err_flag, cudaStream_t st);
+
 // CUDA-core split kernel (any dtype / shape within limits).  Returns
 // cudaErrorNotSupported for shapes it is not built for.
 int simt_grid(const gva_shape_t& sh, int num_sms, long long max_total_tokens, bool gqa);

@@ -74,25 +74,22 @@ template <> struct Vec16<float> {
 // computed before waiting on the preceding kernel (it reads caller inputs only);
 // only the stores of q_abs come after.
 template <typename TQ>
-__global__ void __launch_bounds__(2 * kAbsorbQueries * 32)
-    absorb_query_kernel(int B, int H, int d_h, int d_n, int d_r, float c, const TQ* __restrict__ q,
-                        const TQ* __restrict__ M, const int* __restrict__ q_pos,
-                        float* __restrict__ q_abs, const RopeTable rt, int early_trigger) {
-  extern __shared__ float sm[];
-  // In the fused step the successor (the split kernel) may launch right away: it
-  // waits on this kernel before it reads q_abs, and this kernel waits on the
-  // append before it finishes.
-  if (early_trigger) pdl_trigger();
+__device__ __forceinline__ void absorb_block(int h, int by, int bz, int B, int H, int d_h, int d_n,
+                                             int d_r, float c, const TQ* __restrict__ q,
+                                             const TQ* __restrict__ M,
+                                             const int* __restrict__ q_pos,
+                                             float* __restrict__ q_abs, const RopeTable& rt,
+                                             float* sm, int early_trigger) {
   const int dq = d_n + d_r, dout = d_h + d_r;
-  const int h = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qi = warp % kAbsorbQueries;
-  const int b = blockIdx.y * kAbsorbQueries + qi;
+  const int b = by * kAbsorbQueries + qi;
   float* qv = sm + qi * dq;
   const bool active = b < B;
   const TQ* qrow = q + ((size_t)(active ? b : 0) * H + h) * dq;
   float* o = q_abs + ((size_t)(active ? b : 0) * H + h) * dout;
   if (warp < kAbsorbQueries) {
-    const int i = blockIdx.z * 32 + lane;               // output element of this lane
+    const int i = bz * 32 + lane;                       // output element of this lane
     const bool row_ok = active && i < d_h;
     const TQ* row = M + ((size_t)h * d_h + (row_ok ? i : 0)) * d_n;
     constexpr int V = Vec16<TQ>::N;
@@ -127,7 +124,7 @@ __global__ void __launch_bounds__(2 * kAbsorbQueries * 32)
     if (row_ok) o[i] = (acc0 + acc1) * c;
   } else {
     const int half = d_r / 2;
-    const bool rope = active && blockIdx.z == 0;
+    const bool rope = active && bz == 0;
     const double pos = rope ? (double)q_pos[b] : 0.0;
     double y1[2] = {0.0, 0.0}, y2[2] = {0.0, 0.0};
 #pragma unroll
@@ -150,23 +147,35 @@ __global__ void __launch_bounds__(2 * kAbsorbQueries * 32)
   }
 }
 
+template <typename TQ>
+__global__ void __launch_bounds__(2 * kAbsorbQueries * 32)
+    absorb_query_kernel(int B, int H, int d_h, int d_n, int d_r, float c, const TQ* __restrict__ q,
+                        const TQ* __restrict__ M, const int* __restrict__ q_pos,
+                        float* __restrict__ q_abs, const RopeTable rt, int early_trigger) {
+  extern __shared__ float sm[];
+  // With early_trigger the successor may launch right away: it waits on this
+  // kernel before it reads q_abs.
+  if (early_trigger) pdl_trigger();
+  absorb_block<TQ>(blockIdx.x, blockIdx.y, blockIdx.z, B, H, d_h, d_n, d_r, c, q, M, q_pos, q_abs,
+                   rt, sm, early_trigger);
+}
+
 // One warp per token: the value row is loaded (16-byte vectors) and the
 // positional pairs rotated before waiting on the preceding kernel; the stores
 // into the cache come after.
 template <typename T>
-__global__ void append_cache_kernel(int N, int row_elems, int d_r, const T* __restrict__ v_new,
-                                    const T* __restrict__ kpe_new, const int* __restrict__ slot,
-                                    const int* __restrict__ pos, long long num_slots,
-                                    T* __restrict__ V_cache, T* __restrict__ kr_cache,
-                                    int* __restrict__ err_flag, const RopeTable rt,
-                                    int early_trigger) {
+__device__ __forceinline__ void append_block(long long bx, int N, int row_elems, int d_r,
+                                             const T* __restrict__ v_new,
+                                             const T* __restrict__ kpe_new,
+                                             const int* __restrict__ slot,
+                                             const int* __restrict__ pos, long long num_slots,
+                                             T* __restrict__ V_cache, T* __restrict__ kr_cache,
+                                             int* __restrict__ err_flag, const RopeTable& rt,
+                                             int early_trigger) {
   constexpr int kVecPerLane = 4;   // rows up to 32*4*16 bytes = 2 KB in registers
-  // In the fused step the absorb kernel may launch right away: it writes nothing
-  // this kernel reads, and it waits on this kernel before it finishes.
-  if (early_trigger) pdl_trigger();
   const int warps = blockDim.x >> 5;
   const int lane = threadIdx.x & 31;
-  const long long i = (long long)blockIdx.x * warps + (threadIdx.x >> 5);
+  const long long i = bx * warps + (threadIdx.x >> 5);
   const bool active = i < N;
   const long long s = active ? slot[i] : -1;
   const bool ok = active && s >= 0 && s < num_slots;
@@ -208,6 +217,48 @@ __global__ void append_cache_kernel(int N, int row_elems, int d_r, const T* __re
   }
 }
 
+template <typename T>
+__global__ void append_cache_kernel(int N, int row_elems, int d_r, const T* __restrict__ v_new,
+                                    const T* __restrict__ kpe_new, const int* __restrict__ slot,
+                                    const int* __restrict__ pos, long long num_slots,
+                                    T* __restrict__ V_cache, T* __restrict__ kr_cache,
+                                    int* __restrict__ err_flag, const RopeTable rt,
+                                    int early_trigger) {
+  // With early_trigger the successor may launch right away: it writes nothing
+  // this kernel reads, and it waits on this kernel before it depends on it.
+  if (early_trigger) pdl_trigger();
+  append_block<T>(blockIdx.x, N, row_elems, d_r, v_new, kpe_new, slot, pos, num_slots, V_cache,
+                  kr_cache, err_flag, rt, early_trigger);
+}
+
+// The first two kernels of the fused decode step in one launch: blocks
+// [0, n_absorb) absorb the queries (grid (H, ay, az) flattened), the rest append
+// the new tokens (8 per block).  Each block does its loads and arithmetic, waits
+// on the preceding kernel, then stores.  The successor (the split kernel) may
+// launch at once: it streams only cache rows this kernel does not write before
+// its own wait, and it waits on this kernel before it reads q_abs.
+template <typename TQ, typename T>
+__global__ void __launch_bounds__(256)
+    prep_step_kernel(int n_absorb, int ay, int az, int B, int H, int d_h, int d_n, int d_r,
+                     float c, const TQ* __restrict__ q, const TQ* __restrict__ M,
+                     const int* __restrict__ q_pos, float* __restrict__ q_abs, int N,
+                     int row_elems, const T* __restrict__ v_new, const T* __restrict__ kpe_new,
+                     const int* __restrict__ slot, const int* __restrict__ pos,
+                     long long num_slots, T* __restrict__ V_cache, T* __restrict__ kr_cache,
+                     int* __restrict__ err_flag, const RopeTable rt) {
+  extern __shared__ float sm[];
+  pdl_trigger();
+  const int bid = blockIdx.x;
+  if (bid < n_absorb) {
+    const int per_h = ay * az, r = bid % per_h;
+    absorb_block<TQ>(bid / per_h, r / az, r % az, B, H, d_h, d_n, d_r, c, q, M, q_pos, q_abs, rt,
+                     sm, 1);
+  } else {
+    append_block<T>(bid - n_absorb, N, row_elems, d_r, v_new, kpe_new, slot, pos, num_slots,
+                    V_cache, kr_cache, err_flag, rt, 1);
+  }
+}
+
 static RopeTable rope_table(const gva_shape_t& sh) {
   RopeTable t{};
   for (int i = 0; i < sh.d_r / 2 && i < kMaxRopePairs; ++i)
@@ -236,6 +287,45 @@ cudaError_t launch_absorb(const gva_shape_t& sh, const void* q, const void* M, c
   if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   return launch_pdl(k, grid, block, smem, st, sh.B, sh.H, sh.d_h, sh.d_n, sh.d_r, c, (const float*)q,
                     (const float*)M, q_pos, q_abs, rt, early_trigger ? 1 : 0);
+}
+
+template <typename TQ, typename T>
+static cudaError_t launch_prep_t(const gva_shape_t& sh, const void* q, const void* M,
+                                 const int* q_pos, float* q_abs, float c, int N, const void* v_new,
+                                 const void* kpe_new, const int* slot, const int* pos,
+                                 long long num_slots, void* V_cache, void* kr_cache, int* err_flag,
+                                 cudaStream_t st) {
+  const int ay = (sh.B + kAbsorbQueries - 1) / kAbsorbQueries, az = (sh.d_h + 31) / 32;
+  const int n_absorb = sh.B > 0 ? sh.H * ay * az : 0;
+  const long long n_append = ((long long)N + 7) / 8;     // 256 threads = 8 tokens per block
+  const long long blocks = n_absorb + n_append;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  const size_t smem = sh.B > 0 ? absorb_smem_bytes(sh) : 0;
+  auto k = prep_step_kernel<TQ, T>;
+  if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  return launch_pdl(k, dim3((unsigned)blocks), dim3(256), smem, st, n_absorb, ay, az, sh.B, sh.H,
+                    sh.d_h, sh.d_n, sh.d_r, c, (const TQ*)q, (const TQ*)M, q_pos, q_abs, N,
+                    sh.G * sh.d_h, (const T*)v_new, (const T*)kpe_new, slot, pos, num_slots,
+                    (T*)V_cache, (T*)kr_cache, err_flag, rope_table(sh));
+}
+
+cudaError_t launch_prep_step(const gva_shape_t& sh, const void* q, const void* M, const int* q_pos,
+                             float* q_abs, float c, int N, const void* v_new, const void* kpe_new,
+                             const int* slot, const int* pos, long long num_slots, void* V_cache,
+                             void* kr_cache, int* err_flag, cudaStream_t st) {
+  const bool qb = sh.q_dtype == GVA_BF16, cb = sh.cache_dtype == GVA_BF16;
+  using bf = __nv_bfloat16;
+  if (qb && cb)
+    return launch_prep_t<bf, bf>(sh, q, M, q_pos, q_abs, c, N, v_new, kpe_new, slot, pos,
+                                 num_slots, V_cache, kr_cache, err_flag, st);
+  if (qb)
+    return launch_prep_t<bf, float>(sh, q, M, q_pos, q_abs, c, N, v_new, kpe_new, slot, pos,
+                                    num_slots, V_cache, kr_cache, err_flag, st);
+  if (cb)
+    return launch_prep_t<float, bf>(sh, q, M, q_pos, q_abs, c, N, v_new, kpe_new, slot, pos,
+                                    num_slots, V_cache, kr_cache, err_flag, st);
+  return launch_prep_t<float, float>(sh, q, M, q_pos, q_abs, c, N, v_new, kpe_new, slot, pos,
+                                     num_slots, V_cache, kr_cache, err_flag, st);
 }
 
 cudaError_t launch_append(const gva_shape_t& sh, int N, const void* v_new, const void* kpe_new,
