@@ -353,8 +353,8 @@ def run_ours(args, rank, world, local):
                                  graphs_for, replay, timed, K, dev, row_bytes, part_tokens, ms_dec)
     ms_gqa = None
     if not split_seq:
-        ms_gqa, gqa_bytes = run_gqa_comparison(args, wl, B, H, G, d_h, R, flags, d, graphs_for,
-                                               replay, timed, dev)
+        ms_gqa, gqa_bytes, ms_kv = run_gqa_comparison(args, wl, B, H, G, d_h, R, flags, d,
+                                                      graphs_for, replay, timed, dev)
 
     # end to end through the public API with host buffers: every step copies its
     # inputs (q, new value, new positional key, slot, position) from one pinned
@@ -423,7 +423,10 @@ def run_ours(args, rank, world, local):
             "decode_speedup_vs_gqa": round(ms_gqa / ms_dec, 4),
             "gva_cache_bytes": step_cache_bytes, "gqa_cache_bytes": gqa_bytes,
             "cache_ratio": round(step_cache_bytes / gqa_bytes, 6),
-            "gqa_cache_GBs": round(gqa_bytes / (ms_gqa / K * 1e-3) / 1e9, 2)},
+            "gqa_cache_GBs": round(gqa_bytes / (ms_gqa / K * 1e-3) / 1e9, 2),
+            "shared_kv_decode_steps_per_s": round(K / (ms_kv * 1e-3), 1),
+            "shared_kv_speedup_vs_gqa": round(ms_gqa / ms_kv, 4),
+            "shared_kv_cache_GBs": round(gqa_bytes / 2 / (ms_kv / K * 1e-3) / 1e9, 2)},
         "roofline": {"bound": "hbm",
                      "kernel": ("decode_simt_kernel" if args.fma else "decode_mma_kernel")
                                + " + combine_kernel (one gva_decode_attention call)",
@@ -495,7 +498,24 @@ def run_gqa_comparison(args, wl, B, H, G, d_h, R, flags, d, graphs_for, replay, 
     g_gqa = graphs_for(gqa_decode, args.steps)
     replay(g_gqa)
     ms_gqa, _, _ = timed(g_gqa, args.steps)
-    return ms_gqa, tot_q * 2 * G * d_h * wl.elem_bytes
+    del g_gqa
+
+    # shared keys and values (K = V, the pages' first design): the same batch
+    # with the value cache only, through gva_shared_kv_decode_attention
+    sh_kv = gva.make_shape(B, H, G, d_h, d_h, 0, cache_dtype=wl.torch_dtype, flags=flags,
+                           ctas_per_sm=args.ctas_per_sm)
+    ws_kv = gva.new_workspace(sh_kv, tot_q, device=dev)
+
+    def kv_decode(c):
+        gva.shared_kv_decode_attention(sh_kv, qg, Vq[c], soff_q, slen_q, tot_q, out_q, None, ws_kv)
+
+    for c in range(R):
+        kv_decode(c)
+    g_kv = graphs_for(kv_decode, args.steps)
+    replay(g_kv)
+    ms_kv, _, _ = timed(g_kv, args.steps)
+    assert gva.workspace_status(ws_kv) == 0, "device status word set"
+    return ms_gqa, tot_q * 2 * G * d_h * wl.elem_bytes, ms_kv
 
 
 # ----------------------------------------------------------------------------- oracle arm

@@ -136,7 +136,7 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
                            const int32_t* seq_len, int64_t max_total_tokens, int64_t num_slots,
                            void* out, float* lse, void* workspace, size_t ws_bytes, void* stream,
                            bool prefetch = false, const int32_t* new_slots = nullptr,
-                           int n_new = 0, int nq = 1) {
+                           int n_new = 0, int nq = 1, bool raw_q = false) {
   gva_status_t s = check_shape(shp, gqa);
   if (s != GVA_OK) return s;
   if (nq < 1 || nq > 64) return fail(GVA_ERR_INVALID_ARG, "n_query=%d outside [1,64]", nq);
@@ -175,8 +175,8 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
   a.G = sh.G;
   a.d_h = sh.d_h;
   a.d_r = gqa ? 0 : sh.d_r;
-  a.q_abs = gqa ? nullptr : static_cast<const float*>(q);
-  a.q_raw = gqa ? q : nullptr;
+  a.q_abs = (gqa || raw_q) ? nullptr : static_cast<const float*>(q);
+  a.q_raw = (gqa || raw_q) ? q : nullptr;
   a.q_bf16 = sh.q_dtype == GVA_BF16;
   a.q_scale = scale_of(sh, gqa) * gva::kLog2e;
   a.X = X;
@@ -408,6 +408,21 @@ gva_status_t gva_decode_attention_multi(const gva_shape_t* shape, int32_t n_quer
   return decode_common(shape, false, q_abs, V_cache, V_cache, kr_cache, seq_offset, seq_len,
                        max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream, false,
                        nullptr, 0, n_query);
+}
+
+gva_status_t gva_shared_kv_decode_attention(const gva_shape_t* shape, const void* q,
+                                            const void* V_cache, const int32_t* seq_offset,
+                                            const int32_t* seq_len, int64_t max_total_tokens,
+                                            int64_t num_slots, void* out, float* lse,
+                                            void* workspace, size_t ws_bytes, void* stream) {
+  if (!shape) return fail(GVA_ERR_INVALID_ARG, "shape is NULL");
+  if (shape->d_r != 0 || shape->d_n != shape->d_h)
+    return fail(GVA_ERR_INVALID_ARG, "shared keys and values need d_r == 0 and d_n == d_h (got %d, %d)",
+                shape->d_r, shape->d_n);
+  // keys are the values (M_h = I): the raw query meets the value tile directly
+  return decode_common(shape, false, q, V_cache, V_cache, nullptr, seq_offset, seq_len,
+                       max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream, false,
+                       nullptr, 0, 1, /*raw_q=*/true);
 }
 
 gva_status_t gva_merge_states(const gva_shape_t* shape, int32_t R, const float* outs,

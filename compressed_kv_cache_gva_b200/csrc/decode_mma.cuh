@@ -273,7 +273,9 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       const int vq = hl / hpr, head = g * hpr + hl % hpr;
       float v[C::KS][4];
       float wv[C::RS > 0 ? C::RS : 1][4];
-      if constexpr (!C::GQA) {
+      // absorbed fp32 query (pre-scaled), or the raw query in its storage type,
+      // scaled here: GQA, and GVA with shared keys and values (M = I, d_r = 0)
+      if (!C::GQA && a.q_raw == nullptr) {
         const float* qrow = a.q_abs + (((size_t)b * a.nq + vq) * H + head) * dq;
 #pragma unroll
         for (int ks = 0; ks < C::KS; ++ks) {
@@ -294,7 +296,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
           wv[rs][3] = k0 + 9 < a.d_r ? qrow[C::D_H + k0 + 9] : 0.f;
         }
       } else {
-        const size_t base = ((size_t)b * H + head) * C::D_H;
+        const size_t base = (((size_t)b * a.nq + vq) * H + head) * C::D_H;
 #pragma unroll
         for (int ks = 0; ks < C::KS; ++ks) {
           const int k0 = ks * 16 + 2 * t;
@@ -307,6 +309,10 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
             v[ks][e] = x * a.q_scale;
           }
         }
+#pragma unroll
+        for (int rs = 0; rs < (C::RS > 0 ? C::RS : 1); ++rs)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) wv[rs][e] = 0.f;
       }
       auto part = [&](float x) { const float h = bf16_round(x); return lo ? x - h : h; };
 #pragma unroll

@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(kSimtThreads)
     const long long row0 = __ldg(a.seq_offset + b);
     // query of sequence b, base-2 scaled
     for (int e = tid; e < H * dq; e += blockDim.x) {
-      if (!gqa) {
+      if (!gqa && a.q_raw == nullptr) {
         Qs[e] = a.q_abs[(size_t)b * H * dq + e];
       } else {
         const size_t i = (size_t)b * H * d_h + e;

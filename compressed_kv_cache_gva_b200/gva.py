@@ -93,6 +93,8 @@ def lib() -> ctypes.CDLL:
         L.gva_decode_attention_multi.argtypes = [SP, I32, P, P, P, P, P, I64, I64, P, P, P, SZ, P]
         L.gva_merge_states.restype = ctypes.c_int
         L.gva_merge_states.argtypes = [SP, I32, P, P, P, P, P]
+        L.gva_shared_kv_decode_attention.restype = ctypes.c_int
+        L.gva_shared_kv_decode_attention.argtypes = [SP, P, P, P, P, I64, I64, P, P, P, SZ, P]
         L.gva_decode_attention_noalloc.restype = ctypes.c_int
         L.gva_decode_attention_noalloc.argtypes = [SP, P, P, P, P, P, I64, I64, P, P, P]
         _lib = L
@@ -194,6 +196,15 @@ def decode_attention_multi(shape: Shape, n_query: int, q_abs, V_cache, kr_cache,
         _stream(stream)))
 
 
+def shared_kv_decode_attention(shape: Shape, q, V_cache, seq_offset, seq_len,
+                               max_total_tokens: int, out, lse=None, workspace=None, stream=None):
+    """gva_shared_kv_decode_attention: keys are the values (M_h = I, d_r = 0)."""
+    _check(lib().gva_shared_kv_decode_attention(
+        ctypes.byref(shape), _ptr(q), _ptr(V_cache), _ptr(seq_offset), _ptr(seq_len),
+        int(max_total_tokens), V_cache.shape[0], _ptr(out), _ptr(lse), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
 def merge_states(shape: Shape, outs, lses, out, lse=None, stream=None):
     """gva_merge_states: outs [R,B,H,d_h] float32, lses [R,B,H] float32."""
     _check(lib().gva_merge_states(ctypes.byref(shape), outs.shape[0], _ptr(outs), _ptr(lses),
@@ -216,4 +227,5 @@ def decode_attention_noalloc(shape: Shape, q_abs, V_cache, kr_cache, seq_offset,
 EXPORTS = ["gva_status_string", "gva_last_error", "gva_absorb_query", "gva_append_cache",
            "gva_decode_workspace_size", "gva_decode_attention", "gqa_decode_attention",
            "gva_decode_step", "gva_merge_states", "gva_decode_workspace_size_multi",
-           "gva_decode_attention_multi", "gva_decode_attention_noalloc"]
+           "gva_decode_attention_multi", "gva_decode_attention_noalloc",
+           "gva_shared_kv_decode_attention"]

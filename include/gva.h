@@ -225,6 +225,27 @@ gva_status_t gva_decode_attention_multi(const gva_shape_t* shape, int32_t n_quer
                                         void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * gva_shared_kv_decode_attention — decode with shared keys and values (K = V):
+ * the special case of GVA with M_h = I and no positional slice, the first design
+ * the authors tried, whose cache is exactly half of the matched GQA cache
+ * (onedev.kr review, "How it is used" (어떻게 쓰나)).  Scores s_j = q_h . v_{j,g(h)} / sqrt(d_h),
+ * softmax over the L_b cached rows, o_h = sum_j p_j v_{j,g(h)}.  No absorb step:
+ * the raw query is read in q_dtype and scaled inside the decode kernel.
+ *
+ *   shape      d_r == 0 and d_n == d_h (else GVA_ERR_INVALID_ARG); softmax_scale 0
+ *              -> 1/sqrt(d_h)
+ *   q          device [B, H, d_h] q_dtype (RoPE, if the model uses it, already applied)
+ *   V_cache    device [num_slots, G, d_h] cache_dtype: keys and values
+ *   other arguments, workspace (gva_decode_workspace_size of the same shape),
+ *   alignment and errors as for gva_decode_attention.
+ */
+gva_status_t gva_shared_kv_decode_attention(const gva_shape_t* shape, const void* q,
+                                            const void* V_cache, const int32_t* seq_offset,
+                                            const int32_t* seq_len, int64_t max_total_tokens,
+                                            int64_t num_slots, void* out, float* lse,
+                                            void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * gva_merge_states — merge R attention states of the same queries computed over
  * disjoint parts of each sequence's cache, e.g. one part per GPU when one long
  * sequence's cache is split across GPUs.  The pages have no counterpart (they

@@ -119,3 +119,13 @@ def test_no_device_is_a_cuda_error_not_a_crash(L):
     st = L.gva_decode_attention(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, FAKE, 100, 100, FAKE, None,
                                 FAKE, 1 << 20, None)
     assert st == 4
+
+
+def test_shared_kv_needs_keys_equal_to_values(L):
+    """The shared-KV entry takes only shapes where the keys are the values:
+    no positional slice and a content width equal to the value width."""
+    for bad in (dict(d_r=16), dict(d_n=48, d_r=0)):
+        sh = _shape(**bad)
+        st = L.gva_shared_kv_decode_attention(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, 100, 100,
+                                              FAKE, None, FAKE, 1 << 20, None)
+        assert st == 1 and b"shared keys and values" in L.gva_last_error()
