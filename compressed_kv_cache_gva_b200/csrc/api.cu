@@ -393,10 +393,50 @@ gva_status_t gva_decode_step(const gva_shape_t* shape, const void* q, const void
 
 size_t gva_decode_workspace_size_multi(const gva_shape_t* shape, int32_t n_query,
                                        int64_t max_total_tokens) {
-  if (!shape || n_query < 1 || n_query > 64) return 0;
+  if (!shape || n_query < 1 || shape->G <= 0) return 0;
+  // wide blocks (tcgen05 kernel) write the output directly: only the status word
+  if ((shape->H / shape->G) * (long long)n_query > 8 && !(shape->flags & GVA_FLAG_FMA_PATH))
+    return check_shape(shape, false) == GVA_OK && gva::prefill_supported(*shape, n_query) ? 256 : 0;
+  if (n_query > 64) return 0;
   gva_shape_t shv = *shape;
   shv.H = shape->H * n_query;
   return gva_decode_workspace_size(&shv, max_total_tokens);
+}
+
+// Wide multi-token blocks (more than 8 query columns per value group) run on the
+// tcgen05 kernel: one CTA per 128 query rows of a group, output written directly.
+static gva_status_t prefill_common(const gva_shape_t* shp, int nq, const float* q_abs,
+                                   const void* V_cache, const void* kr_cache,
+                                   const int32_t* seq_offset, const int32_t* seq_len,
+                                   int64_t num_slots, void* out, float* lse, void* workspace,
+                                   size_t ws_bytes, void* stream) {
+  const gva_shape_t& sh = *shp;
+  if (!q_abs || !V_cache || !seq_offset || !seq_len || !out || !workspace)
+    return fail(GVA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (sh.d_r > 0 && !kr_cache) return fail(GVA_ERR_INVALID_ARG, "kr_cache is NULL with d_r > 0");
+  if (!aligned16(q_abs) || !aligned16(V_cache) || (kr_cache && !aligned16(kr_cache)) ||
+      !aligned16(out) || !aligned16(workspace) || !aligned16(seq_offset) || !aligned16(seq_len) ||
+      (lse && !aligned16(lse)))
+    return fail(GVA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (num_slots < 1 || num_slots >= (1ll << 31))
+    return fail(GVA_ERR_INVALID_ARG, "num_slots=%lld outside [1, 2^31)", (long long)num_slots);
+  if (ws_bytes < 4) return fail(GVA_ERR_WORKSPACE, "workspace %zu bytes < 4", ws_bytes);
+  const int row = sh.G * sh.d_h, tt = gva::prefill_tile_rows();
+  CUtensorMap tv{}, tk{};
+  gva_status_t s;
+  if ((s = encode_2d(&tv, V_cache, num_slots, row, row, tt, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != GVA_OK)
+    return s;
+  tk = tv;
+  if (sh.d_r > 0) {
+    const int drp = sh.d_r <= 16 ? 16 : 32;
+    if ((s = encode_2d(&tk, kr_cache, num_slots, sh.d_r, sh.d_r, tt, drp,
+                       drp == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B)) != GVA_OK)
+      return s;
+  }
+  cudaError_t e = gva::launch_prefill(sh, nq, q_abs, seq_offset, seq_len, num_slots, out, lse,
+                                      static_cast<int*>(workspace), tv, tk,
+                                      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GVA_OK : cuda_fail(e, "multi-token tcgen05 kernel launch");
 }
 
 gva_status_t gva_decode_attention_multi(const gva_shape_t* shape, int32_t n_query,
@@ -405,6 +445,18 @@ gva_status_t gva_decode_attention_multi(const gva_shape_t* shape, int32_t n_quer
                                         const int32_t* seq_len, int64_t max_total_tokens,
                                         int64_t num_slots, void* out, float* lse,
                                         void* workspace, size_t ws_bytes, void* stream) {
+  gva_status_t s = check_shape(shape, false);
+  if (s != GVA_OK) return s;
+  if (n_query < 1) return fail(GVA_ERR_INVALID_ARG, "n_query=%d < 1", n_query);
+  if (shape->B == 0) return GVA_OK;
+  if ((shape->H / shape->G) * (long long)n_query > 8 && !(shape->flags & GVA_FLAG_FMA_PATH)) {
+    if (!gva::prefill_supported(*shape, n_query))
+      return fail(GVA_ERR_UNSUPPORTED, "no multi-token kernel for H/G=%d, n_query=%d, d_h=%d, "
+                  "d_r=%d (tcgen05 path: bf16 cache, d_h in {64, 128}, d_r in {0, 8, ..., 32}, "
+                  "H/G dividing 128)", shape->H / shape->G, n_query, shape->d_h, shape->d_r);
+    return prefill_common(shape, n_query, q_abs, V_cache, kr_cache, seq_offset, seq_len,
+                          num_slots, out, lse, workspace, ws_bytes, stream);
+  }
   return decode_common(shape, false, q_abs, V_cache, V_cache, kr_cache, seq_offset, seq_len,
                        max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream, false,
                        nullptr, 0, n_query);

@@ -210,9 +210,17 @@ gva_status_t gva_decode_step(const gva_shape_t* shape, const void* q, const void
  *          B*n_query query tokens (shape->B = B*n_query, q_pos = their positions)
  *   out    device [B, n_query, H, d_h] out_dtype; lse device [B, n_query, H] or NULL
  *   workspace: gva_decode_workspace_size_multi(shape, n_query, max_total_tokens)
- *   Other arguments as gva_decode_attention.  Built for bf16 caches with
- *   (H/G)*n_query in {4, 8} and d_h in {64, 128} (else GVA_ERR_UNSUPPORTED);
- *   n_query = 1 is gva_decode_attention.
+ *   Other arguments as gva_decode_attention.  n_query = 1 is gva_decode_attention.
+ *
+ * Two kernels, by the number of query columns per value group, (H/G)*n_query:
+ *  - 4 or 8 (speculative blocks): the split-KV decode kernel (mma.sync), the
+ *    columns sharing each tile, then the combine; bf16 cache, d_h in {64, 128};
+ *  - more than 8 (chunked prefill, long drafts): the tcgen05 kernel, one CTA per
+ *    128 query rows (token x head) of a group, scores and outputs accumulated in
+ *    tensor memory, output written directly (the workspace only carries the
+ *    status word); bf16 cache, d_h in {64, 128}, d_r a multiple of 8 up to 32,
+ *    H/G dividing 128.
+ * Other shapes return GVA_ERR_UNSUPPORTED.
  */
 size_t gva_decode_workspace_size_multi(const gva_shape_t* shape, int32_t n_query,
                                        int64_t max_total_tokens);

@@ -109,7 +109,7 @@ def test_multi_token_shorter_than_queries():
 
 
 def test_multi_token_unsupported_column_count():
-    wl = WORKLOADS["350m_b8_t4096"]                # H/G = 4: 3 queries make 12 columns
+    wl = WORKLOADS["350m_b8_t4096"].scaled(H=12)   # H/G = 3: 9 columns, 3 does not divide 128
     sh = gva.make_shape(1, wl.H, wl.G, wl.d_h, wl.d_n, wl.d_r)
     d = lambda *s, dt=torch.float32: torch.zeros(*s, dtype=dt, device="cuda")
     ws = torch.zeros(max(gva.decode_workspace_size_multi(sh, 3, 64), 16), dtype=torch.uint8,
