@@ -49,10 +49,12 @@ int num_sms() {
   return cache[dev];
 }
 
-gva_status_t check_shape(const gva_shape_t* sh, bool gqa) {
+// max_b: the decode keeps per-sequence prefix arrays in shared memory (kMaxBatch);
+// the absorb only needs its grid to fit (kMaxQueryRows query rows).
+gva_status_t check_shape(const gva_shape_t* sh, bool gqa, int max_b = gva::kMaxBatch) {
   if (!sh) return fail(GVA_ERR_INVALID_ARG, "shape is NULL");
-  if (sh->B < 0 || sh->B > gva::kMaxBatch)
-    return fail(GVA_ERR_INVALID_ARG, "B=%d outside [0, %d]", sh->B, gva::kMaxBatch);
+  if (sh->B < 0 || sh->B > max_b)
+    return fail(GVA_ERR_INVALID_ARG, "B=%d outside [0, %d]", sh->B, max_b);
   if (sh->H < 1 || sh->G < 1 || sh->H % sh->G)
     return fail(GVA_ERR_INVALID_ARG, "need H >= 1, G >= 1, H %% G == 0 (H=%d G=%d)", sh->H, sh->G);
   if (sh->d_h < 1 || sh->d_h > 512) return fail(GVA_ERR_INVALID_ARG, "d_h=%d outside [1,512]", sh->d_h);
@@ -288,7 +290,7 @@ static gva_status_t append_check(const gva_shape_t& sh, const void* v_new, const
 
 static gva_status_t absorb_impl(const gva_shape_t* shp, const void* q, const void* M,
                                 const int32_t* q_pos, float* q_abs, void* stream, bool early) {
-  gva_status_t s = check_shape(shp, false);
+  gva_status_t s = check_shape(shp, false, gva::kMaxQueryRows);
   if (s != GVA_OK) return s;
   const gva_shape_t& sh = *shp;
   if (sh.B == 0) return GVA_OK;

@@ -17,6 +17,7 @@ namespace gva {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kMaxBatch = 4096;          // sequences per call (prefix array lives in smem)
+constexpr int kMaxQueryRows = 65535 * 4; // query rows of one absorb call (its grid's y extent)
 constexpr uint32_t kWaitLimit = 1u << 22;  // iterations of a bounded mbarrier wait
 
 // ---------------------------------------------------------------------------

@@ -16,7 +16,8 @@
 // of one sequence.  Warp 0 streams 64-token value (and k_rope) tiles with 2-D
 // TMA loads into a ring (no multicast), one thread of warp 1 issues every MMA
 // and owns the tensor memory, warps 4..7 (one TMEM lane quarter each) run the
-// softmax, write P to shared memory and rescale O.  The fp32 query is split into
+// softmax, write P to shared memory (two buffers, so the next tile's softmax
+// overlaps this tile's P.V) and rescale O, lazily.  The fp32 query is split into
 // bf16 hi + lo parts (two MMAs), so the scores keep ~16 bits; P is bf16.
 //
 // Tensor memory (256 columns): S double buffer in columns [0, 64) and [64, 128),
@@ -48,18 +49,18 @@ struct PfCfg {
   static constexpr int CB = D_H / 64;        // 128-byte boxes of a value row
   static constexpr int KS = D_H / 16;        // content k-steps
   static constexpr int RS = DRP / 16;        // positional k-steps
-  static constexpr int STAGES = D_H == 64 ? 4 : 3;
+  static constexpr int STAGES = 3;
   static constexpr int QB = M * D_H * 2;     // q~ hi (or lo): CB boxes of M rows x 128 B
   static constexpr int QRB = DRP ? (M * DRP * 2 + 1023) / 1024 * 1024 : 0;
-  static constexpr int PB = M * TK * 2;      // P: M rows x 128 B
+  static constexpr int PB = M * TK * 2;      // one P buffer: M rows x 128 B (two of them)
   static constexpr int VB = CB * TK * 128;   // value tile of the group
   static constexpr int KRB = DRP ? TK * DRP * 2 : 0;
   static constexpr int STAGE = VB + (KRB + 1023) / 1024 * 1024;
   static constexpr int OFF_Q = 0, OFF_QR = 2 * QB, OFF_P = OFF_QR + 2 * QRB;
-  static constexpr int OFF_RING = OFF_P + PB;
+  static constexpr int OFF_RING = OFF_P + 2 * PB;
   static constexpr int OFF_BAR = OFF_RING + STAGES * STAGE;
-  // full[S], empty[S], s_full[2], s_free[2], p_full, pv_done, fin
-  static constexpr int NBAR = 2 * STAGES + 7;
+  // full[S], empty[S], s_full[2], s_free[2], p_full[2], pv_done[2], fin
+  static constexpr int NBAR = 2 * STAGES + 9;
   static constexpr int SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
   static constexpr uint32_t TMEM_COLS = 256;
   static constexpr uint32_t S_COL = 0, O_COL = 128;
@@ -110,7 +111,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
   const uint32_t full = smem_u32(bars), empty = full + 8 * C::STAGES;
   const uint32_t s_full = empty + 8 * C::STAGES, s_free = s_full + 16;
-  const uint32_t p_full = s_free + 16, pv_done = p_full + 8, fin = pv_done + 8;
+  const uint32_t p_full = s_free + 16, pv_done = p_full + 16, fin = pv_done + 16;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -135,7 +136,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     mbar_init(s_free, 4);
     mbar_init(s_free + 8, 4);
     mbar_init(p_full, 4);
+    mbar_init(p_full + 8, 4);
     mbar_init(pv_done, 1);
+    mbar_init(pv_done + 8, 1);
     mbar_init(fin, 1);
     fence_barrier_init();
     if (blk == 0 && g == 0 && L > 0 && (off < 0 || off + L > a.num_slots))
@@ -250,20 +253,20 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
           tc::commit(s_full + 8 * (k & 1));
         }
-        if (k >= 1) {   // P.V of the previous tile
-          const int kp = k - 1, sp = kp % C::STAGES;
-          ok = ok && mbar_wait(p_full, kp & 1, a.status);
+        if (k >= 1) {   // P.V of the previous tile, P from buffer kp % 2
+          const int kp = k - 1, sp = kp % C::STAGES, pb = kp & 1;
+          ok = ok && mbar_wait(p_full + 8 * pb, (kp >> 1) & 1, a.status);
           tc::fence_after();
           if (ok) {
             const uint32_t vt = sb + C::OFF_RING + sp * C::STAGE;
+            const uint32_t pt = sb + C::OFF_P + pb * C::PB;
 #pragma unroll
             for (int kk = 0; kk < C::TK / 16; ++kk)
-              tc::mma_bf16(tmem + C::O_COL,
-                           tc::smem_desc(sb + C::OFF_P + kk * 32, 16, 1024, tc::kSw128),
+              tc::mma_bf16(tmem + C::O_COL, tc::smem_desc(pt + kk * 32, 16, 1024, tc::kSw128),
                            tc::smem_desc(vt + kk * 16 * 128, C::TK * 128, 1024, tc::kSw128), idO,
                            (kp > 0 || kk > 0) ? 1u : 0u);
           }
-          tc::commit(pv_done);
+          tc::commit(pv_done + 8 * pb);
           tc::commit(empty + 8 * sp);
         }
       }
@@ -298,9 +301,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         s[j] = vis ? s[j] : -INFINITY;
         mx = fmaxf(mx, s[j]);
       }
-      const float mn = fmaxf(m, mx);
+      // Lazy rescaling: a row keeps the max its exponentials are taken against
+      // until a tile's max exceeds it by more than 8 (log2 units), so P <= 2^8 and
+      // O is touched only then.  m = -inf (nothing seen yet) always takes the new max.
+      const bool grow = mx > m + 8.f;
+      const float mn = grow ? mx : m;
       const float ms = mn == -INFINITY ? 0.f : mn;    // no visible key yet: p = 0, alpha = 0
-      const float alpha = ex2(m - ms);
+      const float alpha = ex2(m - ms);                 // 1 when the max is kept
       float rsum = 0.f;
       uint32_t pk[C::TK / 2];
 #pragma unroll
@@ -311,9 +318,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
       l = l * alpha + rsum;
       m = mn;
-      // the P buffer and O are free once the previous P.V has completed
-      if (k >= 1) {
-        ok = ok && mbar_wait(pv_done, (k - 1) & 1, a.status);
+      // P buffer k % 2 is free once the P.V of tile k - 2 has completed
+      const int pb = k & 1;
+      if (k >= 2) {
+        ok = ok && mbar_wait(pv_done + 8 * pb, ((k - 2) >> 1) & 1, a.status);
         tc::fence_after();
       }
       // value rows past the sequence end meet P = 0 but may hold anything (NaN):
@@ -327,14 +335,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
               make_uint4(0, 0, 0, 0);
         }
       }
-      uint8_t* prow = sm + C::OFF_P;
+      uint8_t* prow = sm + C::OFF_P + pb * C::PB;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         *reinterpret_cast<uint4*>(prow + sw128_off(r, c)) =
             make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      // O *= alpha before this tile's P.V accumulates onto it (skipped when no row
-      // of the warp changed its max)
+      // O *= alpha before this tile's P.V accumulates onto it, once the previous
+      // P.V has completed (only when some row of the warp raised its max)
       if (k >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        ok = ok && mbar_wait(pv_done + 8 * ((k - 1) & 1), ((k - 1) >> 1) & 1, a.status);
+        tc::fence_after();
 #pragma unroll
         for (int q4 = 0; q4 < C::D_H / 16; ++q4) {
           float o[16];
@@ -349,10 +359,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       fence_proxy_async_smem();   // P and the zeroed rows are read by the tensor core
       tc::fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(p_full + 8 * pb);
     }
-    if (ntiles > 0) {
-      ok = ok && mbar_wait(pv_done, (ntiles - 1) & 1, a.status);
+    if (ntiles > 0) {   // the last P.V (and with it every earlier one) has completed
+      ok = ok && mbar_wait(pv_done + 8 * ((ntiles - 1) & 1), ((ntiles - 1) >> 1) & 1, a.status);
       tc::fence_after();
     }
     // ---- output: O / l (zero and lse = -inf for a query that sees no cache row)

@@ -91,6 +91,8 @@ const char* gva_last_error(void);
  *            q_abs[b,h,0:d_h]      = c * (q[b,h,0:d_n] @ M[h]^T)
  *            q_abs[b,h,d_h:d_h+d_r]= c * RoPE(q[b,h,d_n:], q_pos[b])
  *          with c = softmax_scale * log2(e)  (scores come out in base-2 units).
+ * Here B counts query rows, up to 262140 (e.g. B * n_query rows for
+ * gva_decode_attention_multi); the decode calls take at most 4096 sequences.
  * Alignment: every pointer 16-byte aligned.  Errors: GVA_ERR_INVALID_ARG.
  */
 gva_status_t gva_absorb_query(const gva_shape_t* shape, const void* q, const void* M,
