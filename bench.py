@@ -52,6 +52,7 @@ def parse():
     p.add_argument("--fma", action="store_true", help="decode on the CUDA-core FMA path")
     p.add_argument("--ctas-per-sm", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-prefill", action="store_true", help="skip the chunked-prefill timing")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--split", default="batch", choices=["batch", "sequence"],
                    help="batch: one independent batch per GPU (weak scaling, default); "
@@ -97,6 +98,16 @@ def load_peaks():
         return float(pk["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def load_peak_record():
+    """The whole measured-peaks record, or None (the bf16 figure falls back to the
+    pool's earlier 1590 TFLOP/s burst measurement)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except Exception:
+        return {"bf16_tflops": 1590.0}
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -347,6 +358,23 @@ def run_ours(args, rank, world, local):
     g_dec = graphs_for(decode_only, K)
     replay(g_dec)
     ms_dec, _, _ = timed(g_dec, K)
+    prefill = None
+    if not args.fma and not split_seq and not args.no_prefill:
+        ms_pf, pf_flops = time_prefill(wl, di, 512, graphs_for, replay, timed, d, dev, K)
+        peaks = load_peak_record()
+        tf_peak = peaks.get("bf16_tflops") if peaks else None
+        tf = pf_flops / (ms_pf * 1e-3) / 1e12
+        prefill = {"n_query": 512, "call": "gva_decode_attention_multi (tcgen05 kernel)",
+                   "tokens_per_sequence": "history + 512",
+                   "us_per_call": round(ms_pf * 1e3, 2), "alg_tflop_per_call": round(pf_flops / 1e12, 4),
+                   "roofline": {"bound": "tensor", "achieved": round(tf, 1),
+                                "peak": tf_peak,
+                                "peak_kind": "measured bf16 burst" if os.path.exists(
+                                    os.path.join(ROOT, "MEASURED_PEAKS.json")) else "fallback",
+                                "unit": "TFLOP/s",
+                                "frac": round(tf / tf_peak, 4) if tf_peak else None,
+                                "flops": "2*(2*d_h + d_r) per (query row, visible key); the kernel "
+                                         "issues ~1.6x that (bf16 hi + lo query halves)"}}
     multi = None
     if not args.fma and not split_seq and (H // G) * 2 in (4, 8):
         multi = time_multi_token(sh, wl, di, 2, Vs, KRs, soff, slen_step, max_total, M, R, d,
@@ -438,6 +466,7 @@ def run_ours(args, rank, world, local):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(ms_e2e / K, 6)},
         "multi_token": multi,
+        "prefill": prefill,
         "gpu_launches": (4 if split_seq else 3) * K,
         "clocks": clocks,
     }
@@ -474,6 +503,48 @@ def time_multi_token(sh, wl, di, Q, Vs, KRs, soff, slen, max_total, M, R, d, gra
     alg = part_tokens * row_bytes + B * Q * H * (d_h + d_r) * 4 + B * Q * H * d_h * 4
     return {"n_query": Q, "call": "gva_decode_attention_multi", "us_per_call": round(s * 1e6, 3),
             "alg_GBs": round(alg / s / 1e9, 2), "time_vs_single_token_decode": round(ms / ms_dec, 4)}
+
+
+def time_prefill(wl, di, Q, graphs_for, replay, timed, d, dev, steps):
+    """Chunked prefill: Q new tokens appended to every sequence of the batch
+    (positions L .. L+Q-1, causal among them), one gva_decode_attention_multi
+    call on the tcgen05 kernel.  Returns the call time and its algorithmic
+    tensor work: per (query row, visible key) 2*(2*d_h + d_r) flops, the scores
+    q~.v + q_r.k_rope and the output p*v."""
+    L = di.seq_len.numpy().astype(np.int64) + Q
+    B, H = len(L), wl.H
+    dq = make_decode_inputs(wl, extra_slots=0, lengths=L)
+    q = make_multi_queries(wl, B, Q)
+    qpos = torch.from_numpy(np.stack([L - Q + i for i in range(Q)], 1).astype(np.int32))
+    sh_q = gva.make_shape(B * Q, H, wl.G, wl.d_h, wl.d_n, wl.d_r, cache_dtype=wl.torch_dtype,
+                          rope_base=wl.rope_base)
+    q_abs = torch.empty(B, Q, H, wl.d_h + wl.d_r, dtype=torch.float32, device=dev)
+    gva.absorb_query(sh_q, d(q.reshape(B * Q, H, -1)), d(dq.M), d(qpos.reshape(-1)), q_abs)
+    sh = gva.make_shape(B, H, wl.G, wl.d_h, wl.d_n, wl.d_r, cache_dtype=wl.torch_dtype,
+                        rope_base=wl.rope_base)
+    tot = int(L.sum())
+    cb = dq.V.numel() * dq.V.element_size() + dq.k_rope.numel() * dq.k_rope.element_size()
+    R = max(2, math.ceil(3 * L2_BYTES / cb))
+    Vs = [d(dq.V) for _ in range(R)]
+    Ks = [d(dq.k_rope) for _ in range(R)]
+    soff, slen = d(dq.seq_offset), d(dq.seq_len)
+    ws = torch.zeros(gva.decode_workspace_size_multi(sh, Q, tot), dtype=torch.uint8, device=dev)
+    out = torch.empty(B, Q, H, wl.d_h, dtype=torch.float32, device=dev)
+
+    def call(c):
+        c %= R   # graphs_for counts copies of the step's cache
+        gva.decode_attention_multi(sh, Q, q_abs, Vs[c], Ks[c], soff, slen, tot, out, None, ws)
+
+    for c in range(R):
+        call(c)
+    n = max(10, min(steps, 200))
+    gs = graphs_for(call, n)
+    replay(gs)
+    ms, _, _ = timed(gs, n)
+    assert gva.workspace_status(ws) == 0, "device status word set"
+    keys = int(sum(Q * (int(l) - Q) + Q * (Q + 1) // 2 for l in L))
+    flops = keys * H * 2 * (2 * wl.d_h + wl.d_r)
+    return ms / n, flops
 
 
 def run_gqa_comparison(args, wl, B, H, G, d_h, R, flags, d, graphs_for, replay, timed, dev):

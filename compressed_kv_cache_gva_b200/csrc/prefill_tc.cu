@@ -124,6 +124,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int rows = min(C::M, nq * hpr - row0);                // valid rows of this block
   const int qi_last = (row0 + rows - 1) / hpr;                 // last query token of the block
   const int kv_end = min(L, L - nq + qi_last + 1);             // keys some row of the block sees
+  const int kv_all = min(L, L - nq + row0 / hpr + 1);          // keys every row of the block sees
   const int ntiles = kv_end > 0 ? (kv_end + C::TK - 1) / C::TK : 0;
 
   if (threadIdx.x == 0) {
@@ -295,11 +296,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (lane == 0) mbar_arrive(s_free + 8 * (k & 1));
       const int t0 = k * C::TK;
       float mx = -INFINITY;
+      if (ok && t0 + C::TK <= kv_all) {   // every row sees the whole tile: no mask
 #pragma unroll
-      for (int j = 0; j < C::TK; ++j) {
-        const bool vis = ok && valid && t0 + j <= lim && t0 + j < L;
-        s[j] = vis ? s[j] : -INFINITY;
-        mx = fmaxf(mx, s[j]);
+        for (int j = 0; j < C::TK; ++j) mx = fmaxf(mx, s[j]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < C::TK; ++j) {
+          const bool vis = ok && valid && t0 + j <= lim && t0 + j < L;
+          s[j] = vis ? s[j] : -INFINITY;
+          mx = fmaxf(mx, s[j]);
+        }
       }
       // Lazy rescaling: a row keeps the max its exponentials are taken against
       // until a tile's max exceeds it by more than 8 (log2 units), so P <= 2^8 and
