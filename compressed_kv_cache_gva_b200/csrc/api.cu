@@ -119,16 +119,24 @@ gva_status_t encode_2d(CUtensorMap* m, const void* base, long long rows, int col
 }
 
 struct Plan {
-  bool mma;
+  bool mma;   // tensor-core split kernel (mma.sync or tcgen05)
+  bool tc;    // the tcgen05 one
   int grid;
   gva::WsLayout ws;
 };
 
-gva_status_t plan_decode(const gva_shape_t& sh, bool gqa, long long max_total, Plan* p) {
+// allow_tc: a one-token GVA decode with an absorbed query, the only case the
+// opt-in tcgen05 kernel covers; multi-token, shared-key and GQA calls always run
+// on the mma.sync kernel.
+gva_status_t plan_decode(const gva_shape_t& sh, bool gqa, long long max_total, Plan* p,
+                         bool allow_tc) {
   const int sms = num_sms();
   if (sms <= 0) return fail(GVA_ERR_CUDA, "no CUDA device");
   p->mma = !(sh.flags & GVA_FLAG_FMA_PATH) && gva::mma_supported(sh, gqa);
-  p->grid = p->mma ? gva::mma_grid(sh, sms, max_total, gqa) : gva::simt_grid(sh, sms, max_total, gqa);
+  p->tc = p->mma && allow_tc && !gqa && (sh.flags & GVA_FLAG_TCGEN05_PATH) &&
+          gva::tc_decode_supported(sh);
+  p->grid = p->tc ? gva::tc_decode_grid(sh, sms, max_total)
+          : p->mma ? gva::mma_grid(sh, sms, max_total, gqa) : gva::simt_grid(sh, sms, max_total, gqa);
   p->ws = gva::ws_layout(sh.B, sh.H, sh.d_h, p->grid);
   return GVA_OK;
 }
@@ -163,7 +171,8 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
     return fail(GVA_ERR_INVALID_ARG, "cache rows must be multiples of 16 bytes (G*d_h*elt=%d, d_r*elt=%d)",
                 sh.G * sh.d_h * e, gqa ? 0 : sh.d_r * e);
   Plan p;
-  if ((s = plan_decode(sh, gqa, max_total_tokens, &p)) != GVA_OK) return s;
+  if ((s = plan_decode(sh, gqa, max_total_tokens, &p, !gqa && !raw_q && nq == 1)) != GVA_OK)
+    return s;
   if (nq > 1 && !p.mma)
     return fail(GVA_ERR_UNSUPPORTED, "several query tokens need the tensor-core kernel "
                 "(bf16 cache, (H/G)*n_query in {4, 8}, d_h in {64, 128})");
@@ -202,7 +211,22 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   cudaError_t err;
-  if (p.mma) {
+  if (p.tc) {
+    a.tile = gva::tc_decode_tile(sh);
+    const int tt = a.tile;
+    const int row = sh.G * sh.d_h;
+    CUtensorMap tv{}, tk{};
+    if ((s = encode_2d(&tv, Vv, num_slots, row, row, tt, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != GVA_OK)
+      return s;
+    tk = tv;
+    if (sh.d_r > 0) {
+      const int drp = sh.d_r <= 16 ? 16 : 32;
+      if ((s = encode_2d(&tk, KR, num_slots, sh.d_r, sh.d_r, tt, drp,
+                         drp == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B)) != GVA_OK)
+        return s;
+    }
+    err = gva::launch_decode_tc(sh, a, tv, tk, st);
+  } else if (p.mma) {
     a.tile = gva::mma_tile(sh, gqa);
     const int tt = a.tile;
     const int row = sh.G * sh.d_h;
@@ -336,9 +360,11 @@ size_t gva_decode_workspace_size(const gva_shape_t* shp, int64_t max_total_token
   size_t best = 0;
   for (int gqa = 0; gqa < 2; ++gqa) {
     if (check_shape(shp, gqa) != GVA_OK) continue;
-    Plan p;
-    if (plan_decode(*shp, gqa, max_total_tokens, &p) != GVA_OK) return 0;
-    if (p.ws.total > best) best = p.ws.total;
+    for (int tc = 0; tc < 2; ++tc) {   // large enough for either split kernel
+      Plan p;
+      if (plan_decode(*shp, gqa, max_total_tokens, &p, tc == 1) != GVA_OK) return 0;
+      if (p.ws.total > best) best = p.ws.total;
+    }
   }
   return best;
 }
@@ -366,7 +392,7 @@ gva_status_t gva_decode_step(const gva_shape_t* shape, const void* q, const void
   if (!q_abs || !V_cache || !seq_offset || !seq_len || !out || !workspace)
     return fail(GVA_ERR_INVALID_ARG, "a required pointer is NULL");
   Plan p;
-  if ((s = plan_decode(*shape, false, max_total_tokens, &p)) != GVA_OK) return s;
+  if ((s = plan_decode(*shape, false, max_total_tokens, &p, true)) != GVA_OK) return s;
   if (ws_bytes < p.ws.total)
     return fail(GVA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, p.ws.total);
   // 1. new tokens into the cache and absorbed queries (one kernel), 2. decode.

@@ -76,6 +76,16 @@ cudaError_t launch_decode_mma(const gva_shape_t& sh, bool gqa, DecodeArgs& a,
                               const CUtensorMap& tm_x, const CUtensorMap& tm_v,
                               const CUtensorMap& tm_kr, cudaStream_t st);
 
+// Opt-in tcgen05 split kernel (decode_tc.cu): one-token GVA decode with H/G = 4, bf16
+// caches, d_h in {64, 128}, G in {4, 8}, d_r <= 32.  Tiles of 128 / G tokens; the
+// value tensor map's box is that many rows x 64 columns, the k_rope map's that
+// many rows x (16 or 32) columns.  Same partials and combine as the mma.sync kernel.
+bool tc_decode_supported(const gva_shape_t& sh);
+int tc_decode_tile(const gva_shape_t& sh);
+int tc_decode_grid(const gva_shape_t& sh, int num_sms, long long max_total_tokens);
+cudaError_t launch_decode_tc(const gva_shape_t& sh, DecodeArgs& a, const CUtensorMap& tm_v,
+                             const CUtensorMap& tm_kr, cudaStream_t st);
+
 // Merge of R normalised states (out, lse) of the same queries (sequence split).
 cudaError_t launch_merge_states(const gva_shape_t& sh, int R, const float* outs, const float* lses,
                                 void* out, float* lse, cudaStream_t st);

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libgva.so")
 
 F32, BF16 = 0, 1
 FLAG_FMA_PATH = 1
+FLAG_TCGEN05_PATH = 2
 DEVERR_RANGE, DEVERR_WAIT = 1, 2
 
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "workspace too small",

@@ -56,6 +56,11 @@ typedef enum { GVA_F32 = 0, GVA_BF16 = 1 } gva_dtype_t;
 
 /* Flags for gva_shape_t.flags. */
 #define GVA_FLAG_FMA_PATH 1u   /* decode on CUDA-core FMA instead of tensor cores  */
+/* One-token GVA decode (H/G = 4, bf16 cache, d_h in {64, 128}, G in {4, 8},
+ * d_r <= 32) on the tcgen05 split kernel instead of the default warp-level
+ * mma.sync one.  Same result to rounding; measured slower on B200 for these thin
+ * products, so it is opt-in.  Ignored for shapes it does not cover. */
+#define GVA_FLAG_TCGEN05_PATH 2u
 
 typedef struct {
   int32_t B;            /* sequences (one query token each)                       */

@@ -111,7 +111,8 @@ def test_append_then_decode_end_to_end():
 
 # ------------------------------------------------------------------ decode
 
-@pytest.mark.parametrize("flags", [0, gva.FLAG_FMA_PATH], ids=["tensor", "fma"])
+@pytest.mark.parametrize("flags", [0, gva.FLAG_TCGEN05_PATH, gva.FLAG_FMA_PATH],
+                         ids=["tensor", "tcgen05", "fma"])
 @pytest.mark.parametrize("name", NAMES)
 def test_decode_matches_oracle(name, flags):
     di = small(name)
@@ -155,6 +156,47 @@ def test_decode_edge_lengths(lengths):
     assert np.all(np.isneginf(lse[L == 0]))
     assert_close(out, ref, "bf16")
     lse_close(lse, ref_lse)
+
+
+@pytest.mark.parametrize("flags", [0, gva.FLAG_TCGEN05_PATH], ids=["tensor", "tcgen05"])
+@pytest.mark.parametrize("name", ["350m_b8_t4096", "dr24_b4_t32768", "d128_b1_t131072"])
+def test_decode_growing_scores(name, flags):
+    """Scores that jump far above everything before them inside one piece: the
+    later rows' values are scaled up, so a row maximum grows by many units of
+    log2 after the first tile (the kernels rescale their accumulated output then).
+    Both orders, growing and shrinking, against the oracle."""
+    di = small(name, lengths=[700, 1500, 90])
+    wl = di.wl
+    V = di.V.float().clone()
+    offs = di.seq_offset.numpy()
+    for b, L in enumerate(di.seq_len.numpy()):
+        L = int(L)
+        ramp = torch.linspace(0.2, 6.0, L) if b != 1 else torch.linspace(6.0, 0.2, L)
+        V[offs[b]:offs[b] + L] *= ramp[:, None, None]
+    di.V = V.to(di.V.dtype)
+    out, lse, _, st = run_gva(di, flags=flags)
+    ref, ref_lse = oracle_gva(di)
+    assert st == 0
+    assert_close(out, ref, wl.dtype, name)
+    lse_close(lse, ref_lse, name)
+
+
+@pytest.mark.parametrize("name", ["350m_b8_t4096", "dr24_b4_t32768", "ragged_b64_1k_16k",
+                                  "d128_b1_t131072"])
+def test_tcgen05_and_mma_sync_kernels_agree(name):
+    """The two tensor-core split kernels (mma.sync, the default, and the opt-in
+    tcgen05 one) compute the same decode; their outputs agree far inside the
+    oracle bar."""
+    di = small(name, lengths=[1, 31, 32, 33, 500, 4097, 16, 17][:max(3, min(8, di_b(name) + 3))])
+    a, la, _, sa = run_gva(di)
+    b, lb, _, sb = run_gva(di, flags=gva.FLAG_TCGEN05_PATH)
+    assert sa == 0 and sb == 0
+    assert np.max(np.abs(a - b)) < 2e-3
+    assert np.max(np.abs(la - lb)) < 2e-3
+
+
+def di_b(name):
+    return WORKLOADS[name].B
 
 
 def test_decode_length_one_returns_the_value_row():

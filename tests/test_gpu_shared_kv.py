@@ -1,7 +1,9 @@
 """Decode with shared keys and values (K = V: M_h = I, d_r = 0) through its own
 entry point, which reads the raw query: against the float64 oracle (the GQA
-oracle with K = V, which the oracle pins show equals GVA with M = I) and
-bit-identical to the absorb route with an identity M."""
+oracle with K = V, which the oracle pins show equals GVA with M = I);
+bit-identical to the absorb route with an identity M on the same (mma.sync)
+split kernel, and within rounding of the absorb route on the opt-in tcgen05
+kernel."""
 import numpy as np
 import pytest
 import torch
@@ -34,7 +36,8 @@ def test_shared_kv_matches_oracle_and_absorb_route(name, lengths):
     q, V = dev(di.q), dev(di.V)
     soff, slen = dev(di.seq_offset), dev(di.seq_len)
     outs = []
-    for route in ("shared", "absorb"):
+    for route in ("shared", "absorb", "absorb-tcgen05"):
+        sh = shape_of(di, flags=gva.FLAG_TCGEN05_PATH if route == "absorb-tcgen05" else 0)
         ws = gva.new_workspace(sh, total)
         out = torch.empty(B, wl.H, wl.d_h, device="cuda")
         lse = torch.empty(B, wl.H, device="cuda")
@@ -55,3 +58,8 @@ def test_shared_kv_matches_oracle_and_absorb_route(name, lengths):
     lse_close(outs[0][1], ref_lse, f"shared-kv {name}")
     assert np.array_equal(outs[0][0], outs[1][0])
     assert np.array_equal(outs[0][1], outs[1][1])
+    assert np.max(np.abs(outs[2][0] - outs[0][0])) < 1e-4
+    a, b = outs[2][1], outs[0][1]
+    assert np.array_equal(np.isneginf(a), np.isneginf(b))     # empty sequences: lse = -inf
+    fin = np.isfinite(b)
+    assert np.max(np.abs(a[fin] - b[fin]), initial=0.0) < 1e-4
