@@ -449,7 +449,7 @@ static gva_status_t prefill_common(const gva_shape_t* shp, int nq, const float* 
   if (num_slots < 1 || num_slots >= (1ll << 31))
     return fail(GVA_ERR_INVALID_ARG, "num_slots=%lld outside [1, 2^31)", (long long)num_slots);
   if (ws_bytes < 4) return fail(GVA_ERR_WORKSPACE, "workspace %zu bytes < 4", ws_bytes);
-  const int row = sh.G * sh.d_h, tt = gva::prefill_tile_rows();
+  const int row = sh.G * sh.d_h, tt = gva::prefill_tile_rows(sh);
   CUtensorMap tv{}, tk{};
   gva_status_t s;
   if ((s = encode_2d(&tv, V_cache, num_slots, row, row, tt, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != GVA_OK)

@@ -28,8 +28,9 @@
 //               d_h = 64 their values stack into the 128 rows of one MMA.
 //
 // Warp roles: warp 0 streams tiles with 2-D TMA loads (no multicast) into a ring,
-// one thread of warp 1 issues every MMA and owns the tensor memory, warps 2-3
-// write each piece's queries (bf16 hi and lo halves) into shared memory, warps
+// one thread of warp 1 issues every MMA and owns the tensor memory, polling for
+// whichever is ready first, the next tile's scores or the next tile's P.V; warps
+// 2-3 write each piece's queries (bf16 hi and lo halves) into shared memory, warps
 // 4-7 (one tensor-memory lane quarter each) run the softmax, write P, rescale O
 // when a row maximum grows by more than 2^8, and store each piece's partial.
 // Every wait is bounded and reported in the status word; the tensor memory is
@@ -56,9 +57,17 @@ struct TcCfg {
   static constexpr int KR1 = TT * DRP * 2;      // one positional box [TT x DRP]
   static constexpr int KRB = G * KR1;           // one copy per group: [group][token][DRP]
   static constexpr int STAGE = VB + KRB;
-  static constexpr int STAGES = 4;
+  static constexpr int MINB = D_H == 64 ? 2 : 1;      // CTAs per SM the budgets are sized for
+  static constexpr int STAGES = (MINB == 2 && DRP == 32) ? 3 : 4;
   static constexpr uint32_t TX = VB + KRB;      // bytes TMA delivers per stage
   static constexpr int NSET = D_H == 64 ? G / 2 : G;   // P.V MMA chains of a tile
+  // Tiles in flight between the roles: the issuer scores up to NSB tiles ahead of
+  // the softmax (score buffers in tensor memory), and the softmax runs up to NPB
+  // tiles ahead of the P.V products (P buffers in shared memory).
+  static constexpr int NPB = 4;
+  static constexpr uint32_t TMEM_LIMIT = MINB == 2 ? 256 : 512;
+  static constexpr int NSB = (4 * NS + NSET * 16 <= (int)TMEM_LIMIT) ? 4
+                           : (3 * NS + NSET * 16 <= (int)TMEM_LIMIT) ? 3 : 2;
   static constexpr int PROW = TT * 2;           // bytes of one P^T row (TT tokens)
   static constexpr int PPAIR = 16 * PROW;       // P^T of one pair of groups
   static constexpr int PBUF = (G / 2) * PPAIR;
@@ -69,18 +78,17 @@ struct TcCfg {
   static constexpr int OFF_Q = OFF_RING + STAGES * STAGE;
   static constexpr int OFF_P = OFF_Q + 2 * QBUF;
   // rescale decisions, by tile parity: tag[2][G] then factors[2][G][4]
-  static constexpr int OFF_RESC = OFF_P + 2 * PBUF;
+  static constexpr int OFF_RESC = OFF_P + NPB * PBUF;
   static constexpr int OFF_BAR = OFF_RESC + (2 * G * 5 * 4 + 15) / 16 * 16;
-  // full[S], empty[S], s_full[2], s_free[2], p_full[2], pv_done[2], q_full[2],
-  // q_free[2], o_free, fin
-  static constexpr int NBAR = 2 * STAGES + 14;
+  // full[STAGES], empty[STAGES], s_full[NSB], s_free[NSB], p_full[NPB], pv_done[NPB],
+  // q_full[2], q_free[2], o_free, fin
+  static constexpr int NBAR = 2 * STAGES + 2 * NSB + 2 * NPB + 6;
   static constexpr int OFF_SCAN = OFF_BAR + NBAR * 8 + 16;
-  static constexpr uint32_t S_COL = 0, O_COL = 2 * NS;
-  static constexpr uint32_t TMEM_NEED = 2 * NS + NSET * 16;
+  static constexpr uint32_t S_COL = 0, O_COL = NSB * NS;
+  static constexpr uint32_t TMEM_NEED = NSB * NS + NSET * 16;
   static constexpr uint32_t TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
-                                      : TMEM_NEED <= 128 ? 128 : 256;
+                                      : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
   static constexpr int THREADS = 256;
-  static constexpr int MINB = D_H == 64 ? 2 : 1;
   static constexpr uint32_t SW_R = DRP == 32 ? tc::kSw64 : tc::kSw32;
   static constexpr uint32_t SBO_R = DRP * 2 * 8;
   static constexpr uint32_t SW_P = TT == 32 ? tc::kSw64 : tc::kSw32;
@@ -88,7 +96,8 @@ struct TcCfg {
   static_assert(G == 4 || G == 8, "groups");
   static_assert(D_H == 64 || D_H == 128, "d_h");
   static_assert(DRP == 0 || DRP == 16 || DRP == 32, "padded d_r");
-  static_assert(TMEM_NEED <= 256, "tensor memory");
+  static_assert(TMEM_NEED <= TMEM_LIMIT && NSB >= 2, "tensor memory");
+  static_assert(NSB + NPB < 16, "issuer ring of tile records");
   static_assert(VB % 1024 == 0 && KR1 % 256 == 0 && PPAIR % 512 == 0, "swizzle atoms");
 
   static size_t smem_bytes(int B) {
@@ -129,6 +138,37 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const float* v) {
       : "memory");
 }
 
+// Non-blocking test of an mbarrier phase (the MMA issuer polls several at once).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Per-tile timeline (-DGVA_TRACE builds only): for the first 8 tiles of each CTA,
+// trace[131072 + (cta * 8 + k) * 8 + which] holds %globaltimer at: 0 tile requested,
+// 1 scores issued, 2 scores seen by the softmax, 3 P buffer free, 4 after the
+// rescale barrier, 5 P handed to the tensor core, 6 P.V issued.
+__device__ __forceinline__ void tc_trace(const DecodeArgs& a, int k, int which) {
+#ifdef GVA_TRACE
+  if (a.trace && k < 8) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    a.trace[131072 + (blockIdx.x * 8 + k) * 8 + which] = t;
+  }
+#else
+  (void)a;
+  (void)k;
+  (void)which;
+#endif
+}
+
 __device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
   asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
@@ -148,8 +188,9 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
   const uint32_t sb = smem_u32(sm);
   const uint32_t bar0 = sb + C::OFF_BAR;
   const uint32_t full = bar0, empty = full + 8 * C::STAGES;
-  const uint32_t s_full = empty + 8 * C::STAGES, s_free = s_full + 16, p_full = s_free + 16;
-  const uint32_t pv_done = p_full + 16, q_full = pv_done + 16, q_free = q_full + 16;
+  const uint32_t s_full = empty + 8 * C::STAGES, s_free = s_full + 8 * C::NSB;
+  const uint32_t p_full = s_free + 8 * C::NSB, pv_done = p_full + 8 * C::NPB;
+  const uint32_t q_full = pv_done + 8 * C::NPB, q_free = q_full + 16;
   const uint32_t o_free = q_free + 16, fin = o_free + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_BAR + C::NBAR * 8);
   int* resc_tag = reinterpret_cast<int*>(sm + C::OFF_RESC);                    // [2][G]
@@ -175,11 +216,15 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       mbar_init(full + 8 * s, 1);
       mbar_init(empty + 8 * s, 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::NSB; ++i) {
       mbar_init(s_full + 8 * i, 1);
       mbar_init(s_free + 8 * i, 4);
+    }
+    for (int i = 0; i < C::NPB; ++i) {
       mbar_init(p_full + 8 * i, 4);
       mbar_init(pv_done + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(q_full + 8 * i, 2);
       mbar_init(q_free + 8 * i, 1);
     }
@@ -217,6 +262,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
   auto issue = [&](int k) {
     const int s = k % C::STAGES;
     const uint32_t fb = full + 8 * s;
+    tc_trace(a, k, 0);
     mbar_arrive_expect_tx(fb, C::TX);
     const uint32_t st = sb + C::OFF_RING + s * C::STAGE;
     const int y = offs[cur.b] + cur.t0;
@@ -291,85 +337,100 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
     if (lane == 0) {
       constexpr uint32_t idS = tc::idesc_bf16(128, C::NS, 0, 0);   // V (K-major) x Qt (K-major)
       constexpr uint32_t idO = tc::idesc_bf16(128, 16, 1, 0);      // V^T (MN-major) x P^T (K-major)
+      const uint64_t dsw128 = tc::smem_desc(0, 16, 1024, tc::kSw128);
+      const uint64_t dswr = tc::smem_desc(0, 16, C::SBO_R, C::SW_R);
+      const uint64_t dv = tc::smem_desc(0, C::D_H == 64 ? C::BOX : C::G * C::BOX, 1024, tc::kSw128);
+      const uint64_t dp = tc::smem_desc(0, 16, C::SBO_P, C::SW_P);
       TileCursor t;
       t.seek(rng, b_first);
-      bool ok = true;
-      int k = 0, n = -1;
-      // the previous tile: its index, its piece, and whether it opened that piece
-      int pk = -1, pn = -1;
-      bool p_first = false;
-      while (true) {
-        const bool have = t.b < a.B;
-        bool first = false;
-        if (have) {
-          int j0, j1;
-          rng.piece(t.b, j0, j1);
-          first = t.t0 == j0;
-          if (first) ++n;
-          const int s = k % C::STAGES;
-          if (first) ok = ok && mbar_wait(q_full + 8 * (n & 1), (n >> 1) & 1, a.status);
-          ok = ok && mbar_wait(full + 8 * s, (k / C::STAGES) & 1, a.status);
-          if (k >= 2) ok = ok && mbar_wait(s_free + 8 * (k & 1), ((k - 2) >> 1) & 1, a.status);
-          tc::fence_after();
-          if (ok) {
-            const uint32_t d = tmem + C::S_COL + (k & 1) * C::NS;
-            const uint32_t vt = sb + C::OFF_RING + s * C::STAGE;
-            const uint32_t qt = sb + C::OFF_Q + (n & 1) * C::QBUF;
+      bool ok = true, scored_all = false;
+      int ks = 0, kp = 0, n = -1;   // next tile to score, next tile to multiply by P
+      // records of the tiles scored but not yet multiplied: whether a tile opened
+      // a piece, and which piece (at most NSB + NPB tiles apart)
+      bool inf_first[16];
+      int inf_piece[16];
+      uint32_t idle = 0;
+      while (ok) {
+        bool progress = false;
+        if (!scored_all) {
+          if (t.b >= a.B) {
+            scored_all = true;
+          } else {
+            int j0, j1;
+            rng.piece(t.b, j0, j1);
+            const bool first = t.t0 == j0;
+            const int nn = first ? n + 1 : n;
+            const int s = ks % C::STAGES, sbuf = ks % C::NSB;
+            const bool ready = (!first || mbar_test(q_full + 8 * (nn & 1), (nn >> 1) & 1)) &&
+                               mbar_test(full + 8 * s, (ks / C::STAGES) & 1) &&
+                               (ks < C::NSB || mbar_test(s_free + 8 * sbuf, ((ks / C::NSB) - 1) & 1));
+            if (ready) {
+              n = nn;
+              tc::fence_after();
+              const uint32_t d = tmem + C::S_COL + sbuf * C::NS;
+              const uint32_t vt = sb + C::OFF_RING + s * C::STAGE;
+              const uint32_t qt = sb + C::OFF_Q + (n & 1) * C::QBUF;
 #pragma unroll
-            for (int ks = 0; ks < C::KS; ++ks) {
-              const uint64_t av = tc::smem_desc(vt + (ks >> 2) * (C::G * C::BOX) + (ks & 3) * 32,
-                                                16, 1024, tc::kSw128);
-              const uint64_t bq = tc::smem_desc(qt + (ks >> 2) * (C::NS * 128) + (ks & 3) * 32,
-                                                16, 1024, tc::kSw128);
-              tc::mma_bf16(d, av, bq, idS, ks > 0);
-            }
+              for (int kx = 0; kx < C::KS; ++kx)
+                tc::mma_bf16(d, dsw128 | ((vt + (kx >> 2) * (C::G * C::BOX) + (kx & 3) * 32) >> 4),
+                             dsw128 | ((qt + (kx >> 2) * (C::NS * 128) + (kx & 3) * 32) >> 4), idS,
+                             kx > 0);
 #pragma unroll
-            for (int rs = 0; rs < C::RS; ++rs) {
-              const uint64_t ak = tc::smem_desc(vt + C::VB + rs * 32, 16, C::SBO_R, C::SW_R);
-              const uint64_t bk = tc::smem_desc(qt + C::QB + rs * 32, 16, C::SBO_R, C::SW_R);
-              tc::mma_bf16(d, ak, bk, idS, 1);
+              for (int rs = 0; rs < C::RS; ++rs)
+                tc::mma_bf16(d, dswr | ((vt + C::VB + rs * 32) >> 4),
+                             dswr | ((qt + C::QB + rs * 32) >> 4), idS, 1);
+              tc::commit(s_full + 8 * sbuf);
+              tc_trace(a, ks, 1);
+              // the queries of this piece are free once its last score MMA completes
+              if (t.t0 + C::TT >= j1) tc::commit(q_free + 8 * (n & 1));
+              inf_first[ks & 15] = first;
+              inf_piece[ks & 15] = n;
+              t.next(rng);
+              ++ks;
+              progress = true;
             }
           }
-          tc::commit(s_full + 8 * (k & 1));
-          // the queries of this piece are free once its last score MMA completes
-          if (t.t0 + C::TT >= j1) tc::commit(q_free + 8 * (n & 1));
         }
-        if (pk >= 0) {
-          // P.V of the previous tile
-          ok = ok && mbar_wait(p_full + 8 * (pk & 1), (pk >> 1) & 1, a.status);
-          // a new piece overwrites O: the previous piece's partial has been read
-          if (p_first && pn >= 1) ok = ok && mbar_wait(o_free, (pn - 1) & 1, a.status);
-          tc::fence_after();
-          if (ok) {
-            const uint32_t vt = sb + C::OFF_RING + (pk % C::STAGES) * C::STAGE;
-            const uint32_t pt = sb + C::OFF_P + (pk & 1) * C::PBUF;
+        if (kp < ks) {
+          const bool jf = inf_first[kp & 15];
+          const int jn = inf_piece[kp & 15], pb = kp % C::NPB;
+          // a new piece overwrites O: the previous piece's partial must have been read
+          const bool ready = mbar_test(p_full + 8 * pb, (kp / C::NPB) & 1) &&
+                             (!(jf && jn >= 1) || mbar_test(o_free, (jn - 1) & 1));
+          if (ready) {
+            tc::fence_after();
+            const uint32_t vt = sb + C::OFF_RING + (kp % C::STAGES) * C::STAGE;
+            const uint32_t pt = sb + C::OFF_P + pb * C::PBUF;
 #pragma unroll
             for (int set = 0; set < C::NSET; ++set) {
               // d_h = 64: the values of groups 2 set, 2 set + 1 fill the 128 rows;
               // d_h = 128: the two 64-column chunks of group `set`
               const int pair = C::D_H == 64 ? set : set / 2;
               const uint32_t abase = C::D_H == 64 ? vt + (2 * set) * C::BOX : vt + set * C::BOX;
-              const uint32_t lbo = C::D_H == 64 ? C::BOX : C::G * C::BOX;
 #pragma unroll
               for (int kk = 0; kk < C::KT; ++kk)
-                tc::mma_bf16(tmem + C::O_COL + set * 16,
-                             tc::smem_desc(abase + kk * 16 * 128, lbo, 1024, tc::kSw128),
-                             tc::smem_desc(pt + pair * C::PPAIR + kk * 32, 16, C::SBO_P, C::SW_P),
-                             idO, (p_first && kk == 0) ? 0u : 1u);
+                tc::mma_bf16(tmem + C::O_COL + set * 16, dv | ((abase + kk * 16 * 128) >> 4),
+                             dp | ((pt + pair * C::PPAIR + kk * 32) >> 4), idO,
+                             (jf && kk == 0) ? 0u : 1u);
             }
+            tc::commit(pv_done + 8 * pb);
+            tc::commit(empty + 8 * (kp % C::STAGES));
+            tc_trace(a, kp, 6);
+            ++kp;
+            progress = true;
           }
-          tc::commit(pv_done + 8 * (pk & 1));
-          tc::commit(empty + 8 * (pk % C::STAGES));
+        } else if (scored_all) {
+          break;   // every tile scored and multiplied
         }
-        if (!have) break;
-        pk = k;
-        pn = n;
-        p_first = first;
-        t.next(rng);
-        ++k;
+        if (progress) {
+          idle = 0;
+        } else if (++idle > 4 * kWaitLimit) {
+          atomicOr(a.status, GVA_DEVERR_WAIT);
+          ok = false;
+        }
       }
       tc::commit(fin);
-      mbar_wait(fin, 0, a.status);
+      mbar_wait(fin, 0, a.status);   // every MMA has completed before the tensor memory is freed
     }
   } else if (warp == 2 || warp == 3) {
     // ---------------------------------------------------------------- queries
@@ -440,76 +501,88 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
     }
     TileCursor t;
     t.seek(rng, b_first);
-    int k = 0, npiece = 0, j0 = 0, j1 = 0;
+    int k = 0, j0 = 0, j1 = 0;
     for (; t.b < a.B; t.next(rng), ++k) {
       rng.piece(t.b, j0, j1);
       const bool first = t.t0 == j0, last = t.t0 + C::TT >= j1;
       const int nvalid = min(C::TT, j1 - t.t0);
       const bool valid = tok < nvalid;
-      ok = ok && mbar_wait(s_full + 8 * (k & 1), (k >> 1) & 1, a.status);
+      const int sbuf = k % C::NSB, pb = k % C::NPB;
+      ok = ok && mbar_wait(s_full + 8 * sbuf, (k / C::NSB) & 1, a.status);
       tc::fence_after();
+      if (threadIdx.x == 128) tc_trace(a, k, 2);
       float sv[8];
       if constexpr (C::TT == 32) {
-        tmem_ld8(lanebase + C::S_COL + (k & 1) * C::NS + g * C::C, sv);
+        tmem_ld8(lanebase + C::S_COL + sbuf * C::NS + g * C::C, sv);
       } else {
         float w16[16];
-        tc::ld16(lanebase + C::S_COL + (k & 1) * C::NS + (2 * q) * C::C, w16);
+        tc::ld16(lanebase + C::S_COL + sbuf * C::NS + (2 * q) * C::C, w16);
 #pragma unroll
         for (int i = 0; i < 8; ++i) sv[i] = lane < 16 ? w16[i] : w16[8 + i];
       }
       tc::wait_ld();
       tc::fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(s_free + 8 * (k & 1));
+      if (lane == 0) mbar_arrive(s_free + 8 * sbuf);
 
-      float s[4], tm[4];
+      const bool live = ok && valid;
+      float s[4];
+      bool ex = false;
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         s[h] = sv[h] + sv[4 + h];
-        tm[h] = (ok && valid) ? s[h] : -INFINITY;
+        ex |= live && s[h] > m_ref[h] + 8.f;
       }
-#pragma unroll
-      for (int o = 1; o < gw; o <<= 1)
-#pragma unroll
-        for (int h = 0; h < 4; ++h) tm[h] = fmaxf(tm[h], __shfl_xor_sync(0xffffffffu, tm[h], o));
+      // The exact maximum over the group's rows is needed on a piece's first tile
+      // and when some row exceeds the reference by more than 8 (log2 units): lazy
+      // rescaling keeps P <= 2^8 otherwise.  The test is warp-uniform, so the
+      // shuffles below always run on the whole warp.
       bool resc = false;
       float alpha[4] = {1.f, 1.f, 1.f, 1.f};
-      if (first) {
+      if (first || __ballot_sync(0xffffffffu, ex) != 0) {
+        float tm[4];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          m_ref[h] = tm[h];
-          l[h] = 0.f;
-        }
-      } else {
-        // lazy rescaling: exponentials stay against m_ref until a tile's max
-        // exceeds it by more than 8 (log2 units), so P <= 2^8
+        for (int h = 0; h < 4; ++h) tm[h] = live ? s[h] : -INFINITY;
 #pragma unroll
-        for (int h = 0; h < 4; ++h)
-          if (tm[h] > m_ref[h] + 8.f) {
-            alpha[h] = ex2(m_ref[h] - tm[h]);
+        for (int o = 1; o < gw; o <<= 1)
+#pragma unroll
+          for (int h = 0; h < 4; ++h) tm[h] = fmaxf(tm[h], __shfl_xor_sync(0xffffffffu, tm[h], o));
+        if (first) {
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
             m_ref[h] = tm[h];
-            l[h] *= alpha[h];
-            resc = true;
+            l[h] = 0.f;
           }
-        if (resc && tok == 0) {
+        } else {
 #pragma unroll
-          for (int h = 0; h < 4; ++h) resc_alpha[((k & 1) * C::G + g) * 4 + h] = alpha[h];
-          resc_tag[(k & 1) * C::G + g] = k + 1;
+          for (int h = 0; h < 4; ++h)
+            if (tm[h] > m_ref[h] + 8.f) {
+              alpha[h] = ex2(m_ref[h] - tm[h]);
+              m_ref[h] = tm[h];
+              l[h] *= alpha[h];
+              resc = true;
+            }
+          if (resc && tok == 0) {
+#pragma unroll
+            for (int h = 0; h < 4; ++h) resc_alpha[((k & 1) * C::G + g) * 4 + h] = alpha[h];
+            resc_tag[(k & 1) * C::G + g] = k + 1;
+          }
         }
       }
       float p[4];
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
-        p[h] = (ok && valid && m_ref[h] != -INFINITY) ? ex2(s[h] - m_ref[h]) : 0.f;
+        p[h] = (live && m_ref[h] != -INFINITY) ? ex2(s[h] - m_ref[h]) : 0.f;
         l[h] += p[h];
       }
-      // P buffer k % 2 is free once the P.V of tile k - 2 has completed
-      if (k >= 2) {
-        ok = ok && mbar_wait(pv_done + 8 * (k & 1), ((k - 2) >> 1) & 1, a.status);
+      // P buffer k % NPB is free once the P.V of tile k - NPB has completed
+      if (k >= C::NPB) {
+        ok = ok && mbar_wait(pv_done + 8 * pb, ((k / C::NPB) - 1) & 1, a.status);
         tc::fence_after();
       }
+      if (threadIdx.x == 128) tc_trace(a, k, 3);
       {
-        const uint32_t pt = sb + C::OFF_P + (k & 1) * C::PBUF + (g >> 1) * C::PPAIR;
+        const uint32_t pt = sb + C::OFF_P + pb * C::PBUF + (g >> 1) * C::PPAIR;
         const int row0 = (g & 1) * 8;
         const int chunk = (tok * 2) >> 4, within = (tok * 2) & 15;
 #pragma unroll
@@ -534,6 +607,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       }
       // all softmax warps see every group's rescale decision of this tile
       named_bar_sync(1, 128);
+      if (threadIdx.x == 128) tc_trace(a, k, 4);
       if (!first) {
         // O lanes this warp owns: d_h = 64: group 2 set + (q >> 1) of every set;
         // d_h = 128: every group (set = group)
@@ -543,7 +617,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
           const int gg = C::D_H == 64 ? 2 * set + (q >> 1) : set;
           if (resc_tag[(k & 1) * C::G + gg] != k + 1) continue;
           if (!waited) {
-            ok = ok && mbar_wait(pv_done + 8 * ((k - 1) & 1), ((k - 1) >> 1) & 1, a.status);
+            // O holds every P.V up to tile k - 1
+            ok = ok && mbar_wait(pv_done + 8 * ((k - 1) % C::NPB), ((k - 1) / C::NPB) & 1, a.status);
             tc::fence_after();
             waited = true;
           }
@@ -560,11 +635,12 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       fence_proxy_async_smem();   // P and zeroed rows are read by the tensor core
       tc::fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full + 8 * (k & 1));
+      if (lane == 0) mbar_arrive(p_full + 8 * pb);
+      if (threadIdx.x == 128) tc_trace(a, k, 5);
 
       if (last) {
         // ---- piece epilogue: (m, l) per head, and O once its last P.V completed
-        ok = ok && mbar_wait(pv_done + 8 * (k & 1), (k >> 1) & 1, a.status);
+        ok = ok && mbar_wait(pv_done + 8 * pb, (k / C::NPB) & 1, a.status);
         tc::fence_after();
 #pragma unroll
         for (int o = 1; o < gw; o <<= 1)
@@ -592,10 +668,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
         tc::fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(o_free);
-        ++npiece;
       }
     }
-    (void)npiece;
   }
 
   // ---- every role is done with the tensor memory: free it

@@ -53,10 +53,10 @@ cudaError_t launch_prep_step(const gva_shape_t& sh, const void* q, const void* M
 
 // Multi-token attention on tcgen05 (prefill_tc.cu): nq new tokens per sequence,
 // causal among them, rows = tokens x heads of a group in blocks of 128.  The
-// value tensor map's box is prefill_tile_rows() x 64, the k_rope map's
-// prefill_tile_rows() x (16 or 32).  Writes out/lse directly (no workspace).
+// value tensor map's box is prefill_tile_rows(sh) x 64, the k_rope map's
+// prefill_tile_rows(sh) x (16 or 32).  Writes out/lse directly (no workspace).
 bool prefill_supported(const gva_shape_t& sh, int nq);
-int prefill_tile_rows();
+int prefill_tile_rows(const gva_shape_t& sh);
 cudaError_t launch_prefill(const gva_shape_t& sh, int nq, const float* q_abs,
                            const int32_t* seq_offset, const int32_t* seq_len, long long num_slots,
                            void* out, float* lse, int* status, const CUtensorMap& tv,

@@ -45,14 +45,21 @@ template <int D_H_, int DRP_>
 struct PfCfg {
   static constexpr int D_H = D_H_, DRP = DRP_;
   static constexpr int M = 128;              // query rows per CTA
-  static constexpr int TK = 64;              // cache tokens per tile (N of the scores)
+  // Cache tokens per tile, the N of the score MMAs.  Each tcgen05 instruction has a
+  // fixed cost well above the arithmetic of a 64-column product, so 128-token tiles
+  // halve the score instructions per key.  With d_h = 128 the CTA's shared memory
+  // allows one CTA per SM either way, and 128-token tiles are 1.5x faster (16384 +
+  // 1024 tokens: 514 vs 776 us on B200).  With d_h = 64, 64-token tiles keep two
+  // CTAs per SM, which hide each other's hand-offs and win (184 vs 216 us for
+  // 8 x (4096 + 512) tokens).
+  static constexpr int TK = D_H == 128 ? 128 : 64;
   static constexpr int CB = D_H / 64;        // 128-byte boxes of a value row
   static constexpr int KS = D_H / 16;        // content k-steps
   static constexpr int RS = DRP / 16;        // positional k-steps
-  static constexpr int STAGES = 3;
+  static constexpr int STAGES = (TK == 128 && D_H == 128) ? 2 : 3;
   static constexpr int QB = M * D_H * 2;     // q~ hi (or lo): CB boxes of M rows x 128 B
   static constexpr int QRB = DRP ? (M * DRP * 2 + 1023) / 1024 * 1024 : 0;
-  static constexpr int PB = M * TK * 2;      // one P buffer: M rows x 128 B (two of them)
+  static constexpr int PB = M * TK * 2;      // one P buffer: TK/64 blocks of M rows x 128 B
   static constexpr int VB = CB * TK * 128;   // value tile of the group
   static constexpr int KRB = DRP ? TK * DRP * 2 : 0;
   static constexpr int STAGE = VB + (KRB + 1023) / 1024 * 1024;
@@ -62,14 +69,16 @@ struct PfCfg {
   // full[S], empty[S], s_full[2], s_free[2], p_full[2], pv_done[2], fin
   static constexpr int NBAR = 2 * STAGES + 9;
   static constexpr int SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
-  static constexpr uint32_t TMEM_COLS = 256;
-  static constexpr uint32_t S_COL = 0, O_COL = 128;
+  static constexpr uint32_t TMEM_COLS = TK == 128 ? 512 : 256;
+  static constexpr uint32_t S_COL = 0, O_COL = 2 * TK;
   static constexpr uint32_t TX = VB + KRB;
   static constexpr int THREADS = 256;
   static constexpr uint32_t SW_R = DRP == 32 ? tc::kSw64 : tc::kSw32;   // k_rope rows of 64 / 32 B
   static constexpr uint32_t SBO_R = DRP * 2 * 8;                         // 8 rows of k_rope
   static_assert(D_H == 64 || D_H == 128, "d_h");
   static_assert(DRP == 0 || DRP == 16 || DRP == 32, "padded d_r");
+  static_assert(TK == 64 || TK == 128, "tile");
+  static_assert(O_COL + D_H <= TMEM_COLS && SMEM <= 227 * 1024, "budgets");
   static_assert(D_H <= 128, "O columns");
 };
 
@@ -263,7 +272,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const uint32_t pt = sb + C::OFF_P + pb * C::PB;
 #pragma unroll
             for (int kk = 0; kk < C::TK / 16; ++kk)
-              tc::mma_bf16(tmem + C::O_COL, tc::smem_desc(pt + kk * 32, 16, 1024, tc::kSw128),
+              tc::mma_bf16(tmem + C::O_COL,
+                           tc::smem_desc(pt + (kk >> 2) * (C::M * 128) + (kk & 3) * 32, 16, 1024,
+                                         tc::kSw128),
                            tc::smem_desc(vt + kk * 16 * 128, C::TK * 128, 1024, tc::kSw128), idO,
                            (kp > 0 || kk > 0) ? 1u : 0u);
           }
@@ -314,22 +325,29 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const float mn = grow ? mx : m;
       const float ms = mn == -INFINITY ? 0.f : mn;    // no visible key yet: p = 0, alpha = 0
       const float alpha = ex2(m - ms);                 // 1 when the max is kept
-      float rsum = 0.f;
-      uint32_t pk[C::TK / 2];
-#pragma unroll
-      for (int j = 0; j < C::TK; j += 2) {
-        const float p0 = ex2(s[j] - ms), p1 = ex2(s[j + 1] - ms);
-        rsum += p0 + p1;
-        pk[j / 2] = pack_bf16(p0, p1);
-      }
-      l = l * alpha + rsum;
-      m = mn;
       // P buffer k % 2 is free once the P.V of tile k - 2 has completed
       const int pb = k & 1;
       if (k >= 2) {
         ok = ok && mbar_wait(pv_done + 8 * pb, ((k - 2) >> 1) & 1, a.status);
         tc::fence_after();
       }
+      // P in bf16, one swizzled 16-byte chunk (8 keys) at a time
+      float rsum = 0.f;
+      uint8_t* prow = sm + C::OFF_P + pb * C::PB;
+#pragma unroll
+      for (int c = 0; c < C::TK / 8; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float p0 = ex2(s[8 * c + 2 * i] - ms), p1 = ex2(s[8 * c + 2 * i + 1] - ms);
+          rsum += p0 + p1;
+          w[i] = pack_bf16(p0, p1);
+        }
+        *reinterpret_cast<uint4*>(prow + (c >> 3) * (C::M * 128) + sw128_off(r, c & 7)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      l = l * alpha + rsum;
+      m = mn;
       // value rows past the sequence end meet P = 0 but may hold anything (NaN):
       // zero them in the last tile before the P.V product reads them
       if (k == ntiles - 1 && t0 + C::TK > L) {
@@ -341,11 +359,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
               make_uint4(0, 0, 0, 0);
         }
       }
-      uint8_t* prow = sm + C::OFF_P + pb * C::PB;
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(prow + sw128_off(r, c)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       // O *= alpha before this tile's P.V accumulates onto it, once the previous
       // P.V has completed (only when some row of the warp raised its max)
       if (k >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
@@ -436,7 +449,7 @@ bool prefill_supported(const gva_shape_t& sh, int nq) {
   return (long long)nq * hpr <= (1ll << 30);
 }
 
-int prefill_tile_rows() { return PfCfg<64, 0>::TK; }
+int prefill_tile_rows(const gva_shape_t& sh) { return sh.d_h == 128 ? PfCfg<128, 0>::TK : PfCfg<64, 0>::TK; }
 
 cudaError_t launch_prefill(const gva_shape_t& sh, int nq, const float* q_abs,
                            const int32_t* seq_offset, const int32_t* seq_len, long long num_slots,

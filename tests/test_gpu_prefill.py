@@ -20,7 +20,9 @@ CASES = [
     (W["350m_b8_t4096"], 32, [1000, 32, 97]),               # 128 rows: one full block
     (W["350m_b8_t4096"], 40, [2049, 64, 41, 300]),          # 160 rows: two blocks
     (W["dr24_b4_t32768"], 24, [777, 130]),                  # d_r = 24 (32-wide positional tile)
-    (W["d128_b1_t131072"], 16, [1500, 16]),                 # d_h = 128
+    (W["d128_b1_t131072"], 16, [1500, 16]),                 # d_h = 128 (128-token tiles)
+    (W["d128_b1_t131072"].scaled(name="d128r24", d_n=104, d_r=24), 40, [300, 129, 1]),
+                                                            # d_h = 128, d_r = 24, two blocks
     (W["350m_b8_t4096"].scaled(name="kv", d_n=64, d_r=0), 33, [500, 66]),   # no positional slice
     (W["350m_b8_t4096"].scaled(name="mha", H=8, G=8), 64, [640, 64]),       # H/G = 1
     (W["350m_b8_t4096"], 5, [3, 0, 7]),                     # sequences shorter than the block
