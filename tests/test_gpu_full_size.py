@@ -45,3 +45,19 @@ def test_full_size_gqa_sampled(name):
     assert st == 0
     assert_close(out[idx], ref[idx], wl.dtype, name)
     lse_close(lse[idx], ref_lse[idx], name)
+
+
+@pytest.mark.parametrize("name", ["350m_b8_t4096", "d128_b1_t131072"])
+def test_full_size_sampled_tcgen05(name):
+    """The opt-in tcgen05 split kernel on the full-size caches, sampled."""
+    from compressed_kv_cache_gva_b200 import gva
+    wl = WORKLOADS[name]
+    di = make_decode_inputs(wl, extra_slots=1)
+    out, lse, _, st = run_gva(di, flags=gva.FLAG_TCGEN05_PATH)
+    pairs = sample_pairs(len(di.seq_len), wl.H, 12 if wl.B > 1 else 6, seed=1)
+    ref, ref_lse = oracle_gva(di, pairs=pairs)
+    idx = tuple(np.array(pairs).T)
+    assert st == 0
+    assert_close(out[idx], ref[idx], wl.dtype, name)
+    lse_close(lse[idx], ref_lse[idx], name)
+    assert np.all(np.isfinite(out))
