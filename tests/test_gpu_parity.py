@@ -146,9 +146,10 @@ def test_decode_split_counts_agree(cps):
 @pytest.mark.parametrize("lengths", [[0], [0, 0, 0], [1], [0, 5, 0, 1], [16, 0, 17], [33] * 9,
                                      [1] * 300], ids=["empty", "all-empty", "one", "mixed-empty",
                                                       "tile-edges", "many-small", "300x1"])
-def test_decode_edge_lengths(lengths):
+@pytest.mark.parametrize("flags", [0, gva.FLAG_TCGEN05_PATH], ids=["tensor", "tcgen05"])
+def test_decode_edge_lengths(lengths, flags):
     di = small("350m_b8_t4096", lengths=lengths)
-    out, lse, _, st = run_gva(di)
+    out, lse, _, st = run_gva(di, flags=flags)
     ref, ref_lse = oracle_gva(di)
     assert st == 0
     L = np.array(lengths)
@@ -208,13 +209,15 @@ def test_decode_length_one_returns_the_value_row():
             np.testing.assert_allclose(out[b, h], V[di.seq_offset[b].item(), h // 4], rtol=0, atol=1e-6)
 
 
-def test_decode_large_batch_scan():
-    """4096 sequences exercise the in-kernel length scan over many threads."""
+@pytest.mark.parametrize("flags", [0, gva.FLAG_TCGEN05_PATH], ids=["tensor", "tcgen05"])
+def test_decode_large_batch_scan(flags):
+    """4096 sequences exercise the in-kernel length scan over many threads, and
+    CTAs that hold many short pieces."""
     rng = np.random.default_rng(3)
     lengths = rng.integers(0, 24, size=4096)
     di = small("350m_b8_t4096", lengths=lengths)
     pairs = [(b, h) for b in rng.choice(4096, 40, replace=False) for h in (0, 7, 15)]
-    out, lse, _, st = run_gva(di)
+    out, lse, _, st = run_gva(di, flags=flags)
     ref, ref_lse = oracle_gva(di, pairs=pairs)
     assert st == 0
     idx = tuple(np.array(pairs).T)
@@ -228,9 +231,10 @@ def test_decode_bf16_output():
     assert_close(out, ref, "bf16")
 
 
-def test_decode_is_deterministic():
+@pytest.mark.parametrize("flags", [0, gva.FLAG_TCGEN05_PATH], ids=["tensor", "tcgen05"])
+def test_decode_is_deterministic(flags):
     di = small("ragged_b64_1k_16k", lengths=[900, 3000, 17, 5000])
-    outs = [run_gva(di)[0] for _ in range(5)]
+    outs = [run_gva(di, flags=flags)[0] for _ in range(5)]
     for o in outs[1:]:
         assert np.array_equal(o, outs[0])
 
