@@ -285,13 +285,20 @@ def test_shared_kv_gva_equals_gqa():
 
 # ------------------------------------------------------------------ fused decode step
 
-@pytest.mark.parametrize("name", ["350m_b8_t4096", "d128_b1_t131072", "tiny_fp32_t64"])
-def test_decode_step_matches_oracle_and_separate_calls(name):
+@pytest.mark.parametrize("name,lengths", [
+    ("350m_b8_t4096", [300, 65, 1, 1031]),
+    ("d128_b1_t131072", [300, 65, 1, 1031]),
+    ("d128_b1_t131072", [3000, 1500]),
+    ("dr24_b4_t32768", [2000, 700, 5]),             # d_r = 24
+    ("350m_b8_t4096", [4096] * 8),                  # the benchmark's batch shape
+    ("tiny_fp32_t64", [300, 65, 1, 1031]),          # fp32 cache: CUDA-core path
+])
+def test_decode_step_matches_oracle_and_separate_calls(name, lengths):
     """gva_decode_step (append, absorb, decode in one call, decode streaming the
     cache before absorb finishes) against the oracle's append + decode, and
     bit-identical to the three separate calls."""
     wl = WORKLOADS[name]
-    lengths = np.array([300, 65, 1, 1031][:max(1, min(4, wl.B + 3))])
+    lengths = np.array(lengths)
     di = make_decode_inputs(wl, extra_slots=1, lengths=lengths)
     V0, K0 = as_f64(di.V), as_f64(di.k_rope)
     offs = di.seq_offset.numpy()
