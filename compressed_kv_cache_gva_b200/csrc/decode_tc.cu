@@ -3,13 +3,13 @@
 //
 // Same work split, partial slots and combine as the default mma.sync split kernel
 // (decode_mma.cuh); the per-tile products run as asynchronous tcgen05 MMAs with
-// fp32 accumulators in tensor memory.  Measured on B200 it is 1.5-2.3x slower than
-// the mma.sync kernel (ncu: tensor pipe ~4% active, warps stalled on barriers and
-// mbarrier waits): a decode tile carries only four exponentials per softmax thread,
-// so the hand-offs between TMA, tensor core and softmax warps set the pace, while
-// the mma.sync kernel keeps a tile's whole dependency chain inside one warp.  It is
-// kept as the measured alternative and as the starting point for a version that
-// moves several tiles per hand-off.
+// fp32 accumulators in tensor memory.  Measured on B200 it is 1.3-1.6x slower than
+// the mma.sync kernel (the first version was 1.5-2.3x slower; ncu: tensor pipe ~4%
+// active, warps stalled on barriers and mbarrier waits): a decode tile carries only
+// four exponentials per softmax thread, so the hand-offs between TMA, tensor core
+// and softmax warps set the pace, while the mma.sync kernel keeps a tile's whole
+// dependency chain inside one warp.  It is kept as the measured alternative and as
+// the starting point for a version that moves several tiles per hand-off.
 //
 // A tile holds TT = 128 / G cache rows, so the G value groups of the tile stack
 // into one 128-row operand: row r = g * TT + t is group g of token t.  Every value
