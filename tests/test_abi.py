@@ -129,3 +129,16 @@ def test_shared_kv_needs_keys_equal_to_values(L):
         st = L.gva_shared_kv_decode_attention(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, 100, 100,
                                               FAKE, None, FAKE, 1 << 20, None)
         assert st == 1 and b"shared keys and values" in L.gva_last_error()
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """No fallback: without the compiled library the binding raises on first use."""
+    import subprocess
+    import sys
+    code = ("from compressed_kv_cache_gva_b200 import gva\n"
+            f"gva.LIB_PATH = {str(tmp_path / 'libgva.so')!r}\n"
+            "gva.lib()\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode != 0
+    assert "is missing" in r.stderr
