@@ -108,19 +108,29 @@ __device__ __forceinline__ void trace_tile(const DecodeArgs& a, int k, int which
 // sequence b form one "piece"; it is written to partial slot i + b.  Two
 // non-empty pieces (b, i) and (b', i') with b + i = b' + i' cannot exist:
 // sequences are contiguous in the tile order, so b' > b forces i' >= i.
+// The grid is sized on the host from an upper bound of the batch's tokens, so it
+// can exceed the batch's tiles.  The split then runs over the first NT CTAs only
+// (one tile each): cut over all of them, some CTAs would own no tile although they
+// sit inside a sequence's run of slots, and the combine would read slots that no
+// CTA wrote.  With NT >= grid, used() == grid and nothing changes.
 // ---------------------------------------------------------------------------
 struct TileSplit {
   int NT;     // tiles in the batch
-  int grid;   // CTAs
-  __device__ __forceinline__ bool narrow() const { return NT <= 0x7fffffff / grid; }
+  int grid;   // CTAs launched
+  // CTAs that own tiles; the rest own none
+  __device__ __forceinline__ int used() const { return grid < NT ? grid : (NT > 0 ? NT : 1); }
+  __device__ __forceinline__ bool narrow() const { return NT <= 0x7fffffff / used(); }
   __device__ __forceinline__ int first(int i) const {
-    return narrow() ? (int)((unsigned)(i * NT) / (unsigned)grid)
-                    : (int)((long long)i * NT / grid);
+    const int g = used();
+    i = i < g ? i : g;
+    return narrow() ? (int)((unsigned)(i * NT) / (unsigned)g)
+                    : (int)((long long)i * NT / g);
   }
   // the CTA that owns tile u (0 <= u < NT): the last i with first(i) <= u
   __device__ __forceinline__ int cta_of(int u) const {
-    return narrow() ? (int)((unsigned)((u + 1) * grid - 1) / (unsigned)NT)
-                    : (int)(((long long)(u + 1) * grid - 1) / NT);
+    const int g = used();
+    return narrow() ? (int)((unsigned)((u + 1) * g - 1) / (unsigned)NT)
+                    : (int)(((long long)(u + 1) * g - 1) / NT);
   }
 };
 
