@@ -1,12 +1,19 @@
 """Benchmark of one GVA decode step on synthetic caches.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--workloads NAME,NAME|none] [--impl ours|reference]
 
-A step is one pass of the whole decode path over one batch: absorb the queries
-(q M^T + query RoPE), append each sequence's new token (value copy + rotated
-positional key), then decode attention over the history plus the new token.
+A step is one pass of the whole decode path over one batch: append each
+sequence's new token (value copy + rotated positional key), absorb the queries
+(q M^T + query RoPE), then decode attention over the history plus the new token.
 Every step reads a different copy of the cache (copies rotate; together they
 exceed 3x the L2), so no step starts with its cache in L2.
+
+Timing: K steps are captured in CUDA graphs; after W warm-up steps the K-step
+pass is replayed back to back until at least 0.2 s (and at least 20 passes) have
+run, with a CUDA event between passes, and the median pass over K is the time
+per step (max over ranks).  The driver's short runs (small K) so measure the same
+steady state as long ones.
 
 Printed: ONE JSON line on rank 0.  value = cache GB/s of the whole job (algorithmic
 cache bytes of all steps on all ranks / max-over-ranks device time).  Under
@@ -16,6 +23,7 @@ path).  `--impl reference` times the float64 CPU oracle on the same workload.
 from __future__ import annotations
 
 import argparse
+import gc
 import hashlib
 import json
 import math
@@ -33,21 +41,30 @@ sys.path.insert(0, ROOT)
 
 from compressed_kv_cache_gva_b200 import gva  # noqa: E402
 from compressed_kv_cache_gva_b200.synth import (WORKLOADS, make_append_inputs,  # noqa: E402
-                                                make_decode_inputs, make_gqa_inputs,
-                                                make_multi_queries)
+                                                make_decode_inputs, make_gqa_append_inputs,
+                                                make_gqa_inputs, make_multi_queries)
 
 METRIC = "GVA decode cache GB/s & %HBM peak (1xB200); decode steps/s vs same-shape GQA"
 DEFAULT_WORKLOAD = "350m_b8_t4096"
+# the long-context workloads of the study, measured in the same run (compact form)
+EXTRA_WORKLOADS = ("dr24_b4_t32768", "ragged_b64_1k_16k", "d128_b1_t131072")
 L2_BYTES = 126 * 1024 * 1024
 NOMINAL_HBM_GBS = 8000.0
+MIN_TIMED_S = 0.2      # every timed measurement replays its K-step pass this long ...
+MIN_PASSES = 20        # ... and at least this many times
+MAX_PASSES = 100000
+CHUNK = 256            # steps per captured graph
 
 
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20000)
-    p.add_argument("--warmup", type=int, default=200)
+    p.add_argument("--steps", type=int, default=1000)
+    p.add_argument("--warmup", type=int, default=50)
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    p.add_argument("--workloads", default=",".join(EXTRA_WORKLOADS),
+                   help="comma-separated workloads also measured (decode, step and GQA "
+                        "comparison), or 'none'")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--fma", action="store_true", help="decode on the CUDA-core FMA path")
     p.add_argument("--ctas-per-sm", type=int, default=0)
@@ -58,7 +75,7 @@ def parse():
                    help="batch: one independent batch per GPU (weak scaling, default); "
                         "sequence: one batch, every sequence's cache split across the GPUs "
                         "(strong scaling, NCCL all-gather + merge)")
-    return p.parse_args()
+    return p.parse_args(argv)
 
 
 def dist_env():
@@ -90,6 +107,13 @@ def job_value(bytes_per_step_per_rank, steps, world, ms_max):
     return world * steps * bytes_per_step_per_rank / (ms_max * 1e-3) / 1e9
 
 
+def passes_for(t_pass_s, min_s=MIN_TIMED_S, min_passes=MIN_PASSES, max_passes=MAX_PASSES):
+    """Number of back-to-back passes of the timed region: at least `min_passes`
+    and at least `min_s` seconds of work."""
+    n = max(min_passes, math.ceil(min_s / max(t_pass_s, 1e-9)))
+    return int(min(n, max_passes))
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -101,13 +125,13 @@ def load_peaks():
 
 
 def load_peak_record():
-    """The whole measured-peaks record, or None (the bf16 figure falls back to the
-    pool's earlier 1590 TFLOP/s burst measurement)."""
+    """The whole measured-peaks record, or the pool's earlier 1590 TFLOP/s bf16
+    burst measurement when it is absent."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            return json.load(f)
+            return json.load(f), "measured bf16 burst"
     except Exception:
-        return {"bf16_tflops": 1590.0}
+        return {"bf16_tflops": 1590.0}, "fallback"
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -152,9 +176,9 @@ class ClockSampler:
 
     def summary(self, t0, t1):
         win = [s for t, s in self.samples if t0 <= t <= t1]
-        label = "timed"
         if len(win) < 3:
             return None
+
         def num(x):
             try:
                 return float(x)
@@ -168,8 +192,84 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(n)
         return {"sm_mhz": float(np.nanmedian(sm)), "sm_max_mhz": num(win[0][3]),
-                "reasons": sorted(reasons), "samples": len(win), "window": label,
+                "reasons": sorted(reasons), "samples": len(win), "window": "timed",
                 "power_w_median": float(np.nanmedian([num(s[4]) for s in win]))}
+
+
+# ----------------------------------------------------------------------------- graphs + timing
+
+class GraphTimer:
+    """Captures K calls of a step function in CUDA graphs (chunks of CHUNK) and
+    times them: the K-step pass is replayed back to back, with an event between
+    passes, for at least MIN_TIMED_S and MIN_PASSES passes; the result is the
+    median pass (max over ranks).  Step i of a pass reads cache copy i mod R."""
+
+    def __init__(self, dev, world):
+        self.dev, self.world = dev, world
+        self.windows = []          # (t0, t1) host times of every timed region
+
+    def capture(self, fn, n, first, R):
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(device=self.dev)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                for i in range(n):
+                    fn((first + i) % R)
+        torch.cuda.current_stream().wait_stream(s)
+        return g
+
+    def graphs(self, fn, K, R):
+        gs, done = [], 0
+        while done < K:
+            n = min(CHUNK, K - done)
+            gs.append((self.capture(fn, n, done, R), n))
+            done += n
+        return gs
+
+    @staticmethod
+    def replay(gs):
+        for g, _ in gs:
+            g.replay()
+
+    def barrier(self):
+        if self.world > 1:
+            torch.distributed.barrier()
+
+    def timed(self, gs):
+        """Median device ms of one pass over `gs` (max over ranks), the number of
+        passes and the host window."""
+        torch.cuda.synchronize()
+        c0 = time.perf_counter()
+        self.replay(gs)                            # calibration pass (untimed)
+        torch.cuda.synchronize()
+        n = passes_for(time.perf_counter() - c0)
+        n = int(reduce_max(n, device=self.dev))    # the same count on every rank
+        st = torch.cuda.current_stream()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+        self.barrier()
+        torch.cuda.synchronize()
+        t0 = time.time()
+        ev[0].record(st)
+        for i in range(n):
+            self.replay(gs)
+            ev[i + 1].record(st)
+        torch.cuda.synchronize()
+        t1 = time.time()
+        self.barrier()
+        per = sorted(ev[i].elapsed_time(ev[i + 1]) for i in range(n))
+        med = per[n // 2] if n % 2 else 0.5 * (per[n // 2 - 1] + per[n // 2])
+        self.windows.append((t0, t1))
+        return reduce_max(med, device=self.dev), n, (t0, t1)
+
+    def time_fn(self, fn, K, R, warm=True):
+        """Capture K steps of fn, warm up, and time them: (ms per step, passes, window)."""
+        gs = self.graphs(fn, K, R)
+        if warm:
+            self.replay(gs)
+        ms, n, win = self.timed(gs)
+        del gs
+        return ms / K, n, win
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -208,193 +308,273 @@ def ncu_traffic(kernel_key, workload):
         return None
 
 
+def copies_for(nbytes):
+    """Cache copies whose total exceeds 3x the L2."""
+    return max(2, math.ceil(3 * L2_BYTES / max(nbytes, 1)))
+
+
+class GQAStep:
+    """The same-shape GQA baseline of a workload: K and V caches (R copies, one
+    free slot per sequence), its decode and its full step (query rotation +
+    append of the new key and value + decode)."""
+
+    def __init__(self, wl, B, flags, ctas_per_sm, dev):
+        d = lambda t: t.to(dev).contiguous()
+        self.gi = gi = make_gqa_inputs(wl, extra_slots=1)
+        L = gi.seq_len.numpy().astype(np.int64)
+        self.B, self.wl = B, wl
+        self.bytes_per_step = int((L + 1).sum()) * 2 * wl.G * wl.d_h * wl.elem_bytes
+        self.R = copies_for(self.bytes_per_step)
+        self.K = [d(gi.K) for _ in range(self.R)]
+        self.V = [d(gi.V) for _ in range(self.R)]
+        kw = dict(cache_dtype=wl.torch_dtype, rope_base=wl.rope_base, flags=flags,
+                  ctas_per_sm=ctas_per_sm)
+        self.sh = gva.make_shape(B, wl.H, wl.G, wl.d_h, wl.d_h, 0, **kw)
+        self.sh_f = gva.make_shape(B, wl.H, wl.G, wl.d_h, wl.d_h, 0, q_dtype=torch.float32, **kw)
+        self.q = d(gi.q)
+        self.q_pos = d(gi.seq_len)
+        self.soff = d(gi.seq_offset)
+        self.slen = d(torch.from_numpy((L + 1).astype(np.int32)))
+        self.total = int((L + 1).sum())
+        ap = make_gqa_append_inputs(wl, (gi.seq_offset.numpy() + L).astype(np.int32),
+                                    L.astype(np.int32))
+        self.k_new, self.v_new, self.slot, self.pos = d(ap.k_new), d(ap.v_new), d(ap.slot), d(ap.pos)
+        self.q_rot = torch.empty(B, wl.H, wl.d_h, dtype=torch.float32, device=dev)
+        self.out = torch.empty(B, wl.H, wl.d_h, dtype=torch.float32, device=dev)
+        self.ws = gva.new_workspace(self.sh, self.total, device=dev)
+
+    def decode(self, c):
+        gva.gqa_decode_attention(self.sh, self.q, self.K[c], self.V[c], self.soff, self.slen,
+                                 self.total, self.out, None, self.ws)
+
+    def step(self, c):
+        gva.gqa_decode_step(self.sh, self.q, self.q_pos, self.k_new, self.v_new, self.slot,
+                            self.pos, self.K[c], self.V[c], self.soff, self.slen, self.total,
+                            self.q_rot, self.out, None, None, self.ws)
+
+    def shared_kv(self, c):
+        gva.shared_kv_decode_attention(self.sh, self.q, self.V[c], self.soff, self.slen,
+                                       self.total, self.out, None, self.ws)
+
+
+class GVAStep:
+    """Buffers and calls of one GVA decode step over one rank's batch."""
+
+    def __init__(self, wl, args, world, rank, dev, split_seq=False):
+        self.wl, self.dev = wl, dev
+        d = lambda t: t.to(dev).contiguous()
+        self.di = di = make_decode_inputs(wl, extra_slots=1)
+        B, H, G, d_h, d_r = len(di.seq_len), wl.H, wl.G, wl.d_h, wl.d_r
+        self.B = B
+        L = di.seq_len.numpy().astype(np.int64)
+        self.row_bytes = cache_row_bytes(wl)
+        self.step_tokens = int((L + 1).sum())                 # history + the appended token
+        self.step_cache_bytes = self.step_tokens * self.row_bytes
+        slots_np = (di.seq_offset.numpy() + L).astype(np.int32)
+        ap = make_append_inputs(wl, slots_np, L.astype(np.int32),
+                                seed=7 + (0 if split_seq else rank))
+        app_host = (ap.v_new, ap.kpe_new, ap.slot, ap.pos)
+        V_src, K_src, soff_src = di.V, di.k_rope, di.seq_offset
+        slen_src = torch.from_numpy((L + 1).astype(np.int32))
+        if split_seq:
+            from compressed_kv_cache_gva_b200 import seqsplit
+            V_src, K_src, soff_src, slen_src, app_host, _ = seqsplit.shard_step_inputs(
+                di.V, di.k_rope, di.seq_offset, L, app_host, world, rank)
+        self.app_host = list(app_host)
+        self.part_tokens = int(slen_src.to(torch.int64).sum())
+        cache_bytes = max(1, V_src.shape[0]) * self.row_bytes
+        self.R = copies_for(cache_bytes)
+        self.l2_note = (f"inputs larger than L2: {self.R} rotating cache copies, "
+                        f"{self.R * cache_bytes / 2**20:.0f} MiB")
+        flags = gva.FLAG_FMA_PATH if args.fma else 0
+        self.flags = flags
+        self.sh = gva.make_shape(B, H, G, d_h, wl.d_n, d_r, cache_dtype=wl.torch_dtype,
+                                 rope_base=wl.rope_base, flags=flags, ctas_per_sm=args.ctas_per_sm)
+        self.Vs = [d(V_src) for _ in range(self.R)]
+        self.KRs = [d(K_src) for _ in range(self.R)]
+        self.q, self.M = d(di.q), d(di.M)
+        self.soff = d(soff_src)
+        self.slen = d(slen_src)
+        self.qpos = d(di.seq_len)                              # new token at position L_b
+        self.v_new, self.kpe_new, self.slot, self.pos = (d(t) for t in self.app_host)
+        self.q_abs = torch.empty(B, H, d_h + d_r, dtype=torch.float32, device=dev)
+        self.out = torch.empty(B, H, d_h, dtype=torch.float32, device=dev)
+        self.max_total = max(self.part_tokens, 1)
+        self.ws = gva.new_workspace(self.sh, self.max_total, device=dev)
+        self.merger = None
+        if split_seq:
+            from compressed_kv_cache_gva_b200 import seqsplit
+            self.merger = seqsplit.SequenceSplitMerge(self.sh, world, dev)
+        self.dec_out = self.merger.out_part if split_seq else self.out
+        self.dec_lse = self.merger.lse_part if split_seq else None
+        # decode-call bytes: cache of this rank + absorbed queries + output
+        self.alg_dec_bytes = (self.part_tokens * self.row_bytes + B * H * (d_h + d_r) * 4
+                              + B * H * d_h * 4)
+
+    def finish(self):
+        if self.merger is not None:
+            self.merger.merge(self.out)
+
+    def step(self, c, qq=None, app=None, o=None):
+        vv, kk, ss, pp = app if app is not None else (self.v_new, self.kpe_new, self.slot, self.pos)
+        gva.decode_step(self.sh, self.q if qq is None else qq, self.M, self.qpos, vv, kk, ss, pp,
+                        self.Vs[c], self.KRs[c], self.soff, self.slen, self.max_total, self.q_abs,
+                        self.dec_out if o is None else o, self.dec_lse, None, self.ws)
+        self.finish()
+
+    def step_separate(self, c):
+        gva.append_cache(self.sh, self.v_new, self.kpe_new, self.slot, self.pos, self.Vs[c],
+                         self.KRs[c])
+        gva.absorb_query(self.sh, self.q, self.M, self.qpos, self.q_abs)
+        gva.decode_attention(self.sh, self.q_abs, self.Vs[c], self.KRs[c], self.soff, self.slen,
+                             self.max_total, self.dec_out, self.dec_lse, self.ws)
+        self.finish()
+
+    def decode_only(self, c):
+        gva.decode_attention(self.sh, self.q_abs, self.Vs[c], self.KRs[c], self.soff, self.slen,
+                             self.max_total, self.dec_out, self.dec_lse, self.ws)
+        self.finish()
+
+
+def decode_figures(st, ms_dec, hbm_peak):
+    """GB/s and roofline fraction of one decode call from its time per call."""
+    s = ms_dec * 1e-3
+    ach = st.alg_dec_bytes / s / 1e9
+    return {"decode_us": round(s * 1e6, 3), "decode_alg_GBs": round(ach, 2),
+            "frac_of_measured": round(ach / hbm_peak, 4),
+            "frac_of_nominal_8TBs": round(ach / NOMINAL_HBM_GBS, 4)}
+
+
+def measure_extra(name, args, timer, sampler, dev, hbm_peak, K):
+    """Compact figures of one more workload: the fused step, the decode call and
+    the same-shape GQA decode and step, each timed like the main workload."""
+    wl = WORKLOADS[name]
+    st = GVAStep(wl, args, 1, 0, dev)
+    for c in range(st.R):
+        st.step(c)
+    torch.cuda.synchronize()
+    t_start = time.time()
+    ms_step, n_step, _ = timer.time_fn(st.step, K, st.R)
+    ms_dec, n_dec, _ = timer.time_fn(st.decode_only, K, st.R)
+    assert gva.workspace_status(st.ws) == 0, f"{name}: device status word set"
+    res = {"B": st.B, "tokens_per_step": st.step_tokens, "cache_bytes_per_step": st.step_cache_bytes,
+           "l2": st.l2_note,
+           "step_us": round(ms_step * 1e3, 3),
+           "step_GBs": round(st.step_cache_bytes / (ms_step * 1e-3) / 1e9, 2),
+           "step_frac_of_measured": round(st.step_cache_bytes / (ms_step * 1e-3) / 1e9 / hbm_peak, 4)}
+    res.update(decode_figures(st, ms_dec, hbm_peak))
+    B = st.B
+    del st
+    gc.collect()
+    torch.cuda.empty_cache()
+    if not args.fma:
+        gq = GQAStep(wl, B, 0, args.ctas_per_sm, dev)
+        for c in range(gq.R):
+            gq.step(c)
+        ms_gd, _, _ = timer.time_fn(gq.decode, K, gq.R)
+        ms_gs, _, _ = timer.time_fn(gq.step, K, gq.R)
+        assert gva.workspace_status(gq.ws) == 0, f"{name}: GQA status word set"
+        res.update({"gqa_decode_us": round(ms_gd * 1e3, 3),
+                    "decode_speedup_vs_gqa": round(ms_gd / ms_dec, 4),
+                    "gqa_step_us": round(ms_gs * 1e3, 3),
+                    "step_speedup_vs_gqa": round(ms_gs / ms_step, 4),
+                    "gqa_cache_bytes_per_step": gq.bytes_per_step})
+        del gq
+        gc.collect()
+        torch.cuda.empty_cache()
+    res["passes"] = {"step": n_step, "decode": n_dec}
+    res["clocks"] = sampler.summary(t_start, time.time())
+    return res
+
+
 def run_ours(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     split_seq = args.split == "sequence"
     # sequence split: every rank holds a part of the same batch
     wl = WORKLOADS[args.workload] if split_seq else rank_workload(args.workload, rank)
-    di = make_decode_inputs(wl, extra_slots=1)
-    B, H, G, d_h, d_r = len(di.seq_len), wl.H, wl.G, wl.d_h, wl.d_r
-    L = di.seq_len.numpy().astype(np.int64)
-    row_bytes = cache_row_bytes(wl)
-    step_tokens = int((L + 1).sum())                       # history + the appended token
-    step_cache_bytes = step_tokens * row_bytes             # this rank's batch (or whole batch)
-    slots_np = (di.seq_offset.numpy() + L).astype(np.int32)
-    ap = make_append_inputs(wl, slots_np, L.astype(np.int32), seed=7 + (0 if split_seq else rank))
-    app_host = [ap.v_new, ap.kpe_new, ap.slot, ap.pos]
-    V_src, K_src, soff_src = di.V, di.k_rope, di.seq_offset
-    slen_src = torch.from_numpy((L + 1).astype(np.int32))
-    if split_seq:
-        from compressed_kv_cache_gva_b200 import seqsplit
-        V_src, K_src, soff_src, slen_src, start = seqsplit.shard_cache(
-            di.V, di.k_rope, di.seq_offset, slen_src, world, rank)
-        cnt = slen_src.numpy().astype(np.int64)
-        own = (L >= start) & (L < start + cnt)            # new token of sequence b lands here
-        sl = (soff_src.numpy().astype(np.int64) + L - start)[own].astype(np.int32)
-        app_host = [ap.v_new[torch.from_numpy(own)].contiguous(),
-                    ap.kpe_new[torch.from_numpy(own)].contiguous(),
-                    torch.from_numpy(sl), ap.pos[torch.from_numpy(own)].contiguous()]
-    part_tokens = int(slen_src.to(torch.int64).sum())
-    cache_bytes = max(1, V_src.shape[0]) * row_bytes
-    R = max(2, math.ceil(3 * L2_BYTES / cache_bytes))
-    flags = gva.FLAG_FMA_PATH if args.fma else 0
-    sh = gva.make_shape(B, H, G, d_h, wl.d_n, d_r, cache_dtype=wl.torch_dtype, rope_base=wl.rope_base,
-                        flags=flags, ctas_per_sm=args.ctas_per_sm)
+    st = GVAStep(wl, args, world, rank, dev, split_seq=split_seq)
+    B, H, G, d_h, d_r = st.B, wl.H, wl.G, wl.d_h, wl.d_r
+    R = st.R
+    timer = GraphTimer(dev, world)
+    K, W = args.steps, max(args.warmup, 3)
 
-    d = lambda t: t.to(dev).contiguous()
-    Vs = [d(V_src) for _ in range(R)]
-    KRs = [d(K_src) for _ in range(R)]
-    q, M = d(di.q), d(di.M)
-    soff = d(soff_src)
-    slen_step = d(slen_src)
-    qpos = d(di.seq_len)                                    # new token at position L_b
-    v_new, kpe_new, slot, pos = (d(t) for t in app_host)
-    q_abs = torch.empty(B, H, d_h + d_r, dtype=torch.float32, device=dev)
-    out = torch.empty(B, H, d_h, dtype=torch.float32, device=dev)
-    max_total = max(part_tokens, 1)
-    ws = gva.new_workspace(sh, max_total, device=dev)
-    merger = None
-    if split_seq:
-        merger = seqsplit.SequenceSplitMerge(sh, world, dev)
-    dec_out = merger.out_part if split_seq else out
-    dec_lse = merger.lse_part if split_seq else None
-
-    def finish():
-        if split_seq:
-            merger.merge(out)
-
-    def step(c, qq=None, app=None, o=None):
-        vv, kk, ss, pp = app if app is not None else (v_new, kpe_new, slot, pos)
-        gva.decode_step(sh, q if qq is None else qq, M, qpos, vv, kk, ss, pp, Vs[c], KRs[c], soff,
-                        slen_step, max_total, q_abs, dec_out if o is None else o, dec_lse, None, ws)
-        finish()
-
-    def step_separate(c):
-        gva.append_cache(sh, v_new, kpe_new, slot, pos, Vs[c], KRs[c])
-        gva.absorb_query(sh, q, M, qpos, q_abs)
-        gva.decode_attention(sh, q_abs, Vs[c], KRs[c], soff, slen_step, max_total, dec_out, dec_lse,
-                             ws)
-        finish()
-
-    def decode_only(c):
-        gva.decode_attention(sh, q_abs, Vs[c], KRs[c], soff, slen_step, max_total, dec_out, dec_lse,
-                             ws)
-        finish()
-
-    # eager warm-up (initialises the library and the launch attributes)
+    # eager warm-up (initialises the library and every cache copy)
     for c in range(R):
-        step(c)
+        st.step(c)
     torch.cuda.synchronize()
 
-    def capture(fn, n, first=0):
-        g = torch.cuda.CUDAGraph()
-        s = torch.cuda.Stream(device=dev)
-        s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s):
-            with torch.cuda.graph(g, stream=s):
-                for i in range(n):
-                    fn((first + i) % R)
-        torch.cuda.current_stream().wait_stream(s)
-        return g
-
-    CHUNK = 256
-
-    def graphs_for(fn, K):
-        gs = []
-        done = 0
-        while done < K:
-            n = min(CHUNK, K - done)
-            gs.append((capture(fn, n, done), n))
-            done += n
-        return gs
-
-    def replay(gs):
-        for g, _ in gs:
-            g.replay()
-
-    def timed(gs, K, sampler_window=None):
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize()
-        st = torch.cuda.current_stream()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        t0 = time.time()
-        e0.record(st)
-        replay(gs)
-        e1.record(st)
-        torch.cuda.synchronize()
-        t1 = time.time()
-        if world > 1:
-            torch.distributed.barrier()
-        ms = reduce_max(e0.elapsed_time(e1), device=dev)
-        return ms, t0, t1
-
-    K, W = args.steps, args.warmup
-    g_warm = graphs_for(step, max(W, 1))
-    g_time = graphs_for(step, K)
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.2)
+    g_warm = timer.graphs(st.step, W, R)
+    g_time = timer.graphs(st.step, K, R)
     tw0 = time.time()
-    replay(g_warm)
+    timer.replay(g_warm)
     torch.cuda.synchronize()
-    ms, t0, t1 = timed(g_time, K)
+    ms_pass, n_pass, (t0, t1) = timer.timed(g_time)
     clocks = sampler.summary(tw0, t1)
-    if clocks is None:
-        # timed region too short for 50 ms sampling: keep the same graphs running
-        # (untimed) for about a second and report the clocks seen under that load
-        s0 = time.time()
-        while time.time() - s0 < 1.2:
-            replay(g_time)
-            torch.cuda.synchronize()
-        clocks = sampler.summary(tw0, time.time())
-        if clocks is not None:
-            clocks["window"] = "warm-up + timed + untimed soak of the same step graphs"
-    sampler.stop()
-    assert gva.workspace_status(ws) == 0, "device status word set"
+    del g_warm, g_time
+    assert gva.workspace_status(st.ws) == 0, "device status word set"
+    ms_step = ms_pass / K
 
     # the same step as three separate calls (no early cache streaming), for reference
-    g_sep = graphs_for(step_separate, K)
-    replay(g_sep)
-    ms_sep, _, _ = timed(g_sep, K)
-    del g_sep
+    ms_sep, _, _ = timer.time_fn(st.step_separate, K, R)
+    # decode-only timing (roofline of the dominant kernel)
+    ms_dec, n_dec, _ = timer.time_fn(st.decode_only, K, R)
 
-    # decode-only timing (roofline of the dominant kernel) and the GQA comparison
-    g_dec = graphs_for(decode_only, K)
-    replay(g_dec)
-    ms_dec, _, _ = timed(g_dec, K)
+    hbm_peak, peak_kind = load_peaks()
     prefill = None
     if not args.fma and not split_seq and not args.no_prefill:
-        ms_pf, pf_flops = time_prefill(wl, di, 512, graphs_for, replay, timed, d, dev, K)
-        peaks = load_peak_record()
-        tf_peak = peaks.get("bf16_tflops") if peaks else None
+        ms_pf, pf_flops = time_prefill(wl, st.di, 512, timer, dev, K)
+        peaks, pk_kind = load_peak_record()
+        tf_peak = peaks.get("bf16_tflops")
         tf = pf_flops / (ms_pf * 1e-3) / 1e12
         prefill = {"n_query": 512, "call": "gva_decode_attention_multi (tcgen05 kernel)",
                    "tokens_per_sequence": "history + 512",
                    "us_per_call": round(ms_pf * 1e3, 2), "alg_tflop_per_call": round(pf_flops / 1e12, 4),
-                   "roofline": {"bound": "tensor", "achieved": round(tf, 1),
-                                "peak": tf_peak,
-                                "peak_kind": "measured bf16 burst" if os.path.exists(
-                                    os.path.join(ROOT, "MEASURED_PEAKS.json")) else "fallback",
-                                "unit": "TFLOP/s",
+                   "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": tf_peak,
+                                "peak_kind": pk_kind, "unit": "TFLOP/s",
                                 "frac": round(tf / tf_peak, 4) if tf_peak else None,
                                 "flops": "2*(2*d_h + d_r) per (query row, visible key); the kernel "
                                          "issues ~1.6x that (bf16 hi + lo query halves)"}}
     multi = None
     if not args.fma and not split_seq and (H // G) * 2 in (4, 8):
-        multi = time_multi_token(sh, wl, di, 2, Vs, KRs, soff, slen_step, max_total, M, R, d,
-                                 graphs_for, replay, timed, K, dev, row_bytes, part_tokens, ms_dec)
-    ms_gqa = None
-    if not split_seq:
-        ms_gqa, gqa_bytes, ms_kv = run_gqa_comparison(args, wl, B, H, G, d_h, R, flags, d,
-                                                      graphs_for, replay, timed, dev)
+        multi = time_multi_token(st, 2, timer, K, dev, ms_dec)
+    gqa_cmp = None
+    if not split_seq and not args.fma:
+        gq = GQAStep(wl, B, 0, args.ctas_per_sm, dev)
+        for c in range(gq.R):
+            gq.step(c)
+        ms_gd, _, _ = timer.time_fn(gq.decode, K, gq.R)
+        ms_gs, _, _ = timer.time_fn(gq.step, K, gq.R)
+        ms_kv, _, _ = timer.time_fn(gq.shared_kv, K, gq.R)
+        assert gva.workspace_status(gq.ws) == 0, "GQA status word set"
+        gb = gq.bytes_per_step
+        gqa_cmp = {
+            "gva_decode_steps_per_s": round(1e3 / ms_dec, 1),
+            "gqa_decode_steps_per_s": round(1e3 / ms_gd, 1),
+            "decode_speedup_vs_gqa": round(ms_gd / ms_dec, 4),
+            "gva_full_steps_per_s": round(1e3 / ms_step, 1),
+            "gqa_full_steps_per_s": round(1e3 / ms_gs, 1),
+            "full_step_speedup": round(ms_gs / ms_step, 4),
+            "gqa_full_step": "gqa_decode_step: query rotation + append of key and value (one "
+                             "kernel), GQA decode (split + combine)",
+            "gva_cache_bytes": st.step_cache_bytes, "gqa_cache_bytes": gb,
+            "cache_ratio": round(st.step_cache_bytes / gb, 6),
+            "gqa_cache_GBs": round(gb / (ms_gd * 1e-3) / 1e9, 2),
+            "shared_kv_decode_steps_per_s": round(1e3 / ms_kv, 1),
+            "shared_kv_speedup_vs_gqa": round(ms_gd / ms_kv, 4),
+            "shared_kv_cache_GBs": round(gb / 2 / (ms_kv * 1e-3) / 1e9, 2)}
+        del gq
+        gc.collect()
+        torch.cuda.empty_cache()
 
     # end to end through the public API with host buffers: every step copies its
     # inputs (q, new value, new positional key, slot, position) from one pinned
     # host buffer into one device staging buffer, runs the step on views of it,
     # and reads the output back into pinned host memory
-    parts = [di.q] + app_host
+    parts = [st.di.q] + st.app_host
     offs_b, nb = [], 0
     for t in parts:
         offs_b.append(nb)
@@ -416,29 +596,30 @@ def run_ours(args, rank, world, local):
 
     def e2e_step(c):
         d_stage.copy_(h_stage, non_blocking=True)
-        step(c, qq=eq, app=(ev, ek, es, ep))
-        h_out.copy_(out, non_blocking=True)
+        st.step(c, qq=eq, app=(ev, ek, es, ep))
+        h_out.copy_(st.out, non_blocking=True)
 
-    g_e2e = graphs_for(e2e_step, K)
-    replay(g_e2e)
-    ms_e2e_serial, _, _ = timed(g_e2e, K)
-    del g_e2e
+    ms_e2e_serial, _, _ = timer.time_fn(e2e_step, K, R)
     ms_e2e = ms_e2e_serial
     e2e_mode = "serial: copy in, step, copy out, one after the other on one stream"
     if not split_seq:
-        ms_e2e = time_e2e_pipelined(step, parts, h_stage, nb, view, B, H, d_h, R, K, dev, timed)
+        ms_e2e = time_e2e_pipelined(st, parts, h_stage, nb, view, K, dev, timer)
         e2e_mode = ("pipelined: every step copies its inputs host->device and its output "
                     "device->host on two copy streams, through two staging and output buffers, "
                     "so the copies of one step overlap the compute of its neighbours")
 
-    hbm_peak, peak_kind = load_peaks()
-    ms_step = ms / K
+    workloads = {}
+    extra = [] if (args.workloads in ("", "none") or split_seq or world > 1) else \
+        [w for w in args.workloads.split(",") if w and w != wl.name]
+    for name in extra:
+        workloads[name] = measure_extra(name, args, timer, sampler, dev, hbm_peak, K)
+    sampler.stop()
+
     job_ranks = 1 if split_seq else world      # sequence split: one batch for all ranks
-    value = job_value(step_cache_bytes, K, job_ranks, ms)
-    dec_s = ms_dec / K * 1e-3
-    alg_dec_bytes = part_tokens * row_bytes + B * H * (d_h + d_r) * 4 + B * H * d_h * 4
-    achieved = alg_dec_bytes / dec_s / 1e9
+    value = job_value(st.step_cache_bytes, 1, job_ranks, ms_step)
+    dec = decode_figures(st, ms_dec, hbm_peak)
     kernel_key = "gva_decode_attention" + ("_fma" if args.fma else "")
+    launches_per_step = 4 if split_seq else 3
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": round(ms_step, 6), "higher_is_better": True,
@@ -446,51 +627,47 @@ def run_ours(args, rank, world, local):
         "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": wl.name, "B": B, "H": H, "G": G, "d_h": d_h, "d_n": wl.d_n, "d_r": d_r,
                    "T": wl.T, "ragged": wl.ragged, "rope_base": wl.rope_base,
-                   "tokens_per_step": step_tokens, "cache_bytes_per_step": step_cache_bytes,
-                   "l2": f"inputs larger than L2: {R} rotating cache copies, "
-                         f"{R * cache_bytes / 2**20:.0f} MiB",
+                   "tokens_per_step": st.step_tokens, "cache_bytes_per_step": st.step_cache_bytes,
+                   "l2": st.l2_note,
                    "parallelism": (f"sequence split: each sequence's cache over {world} GPU(s), "
                                    "NCCL all-gather of (out, lse) + merge") if split_seq else
                                   f"weak: {world} independent batch(es), one per GPU",
                    "step": "gva_decode_step: append + absorb (one kernel), decode (split + combine)",
-                   "graphs": "CUDA graphs",
+                   "graphs": "CUDA graphs of the K steps; the K-step pass replayed back to back, "
+                             "median pass",
                    "decode_path": "fma" if args.fma else "tensor"},
-        "steps_per_s": round(world * K / (ms * 1e-3), 1),
-        "ms_per_step_separate_calls": round(ms_sep / K, 6),
+        "timing": {"passes": n_pass, "timed_region_s": round(t1 - t0, 3),
+                   "ms_per_pass_median": round(ms_pass, 6), "min_timed_s": MIN_TIMED_S,
+                   "min_passes": MIN_PASSES},
+        "steps_per_s": round(world * 1e3 / ms_step, 1),
+        "ms_per_step_separate_calls": round(ms_sep, 6),
         "pct_hbm_peak": {"of_measured": round(value / world / hbm_peak, 4),
                          "of_nominal_8TBs": round(value / world / NOMINAL_HBM_GBS, 4)},
-        "gqa_comparison": None if ms_gqa is None else {
-            "gva_decode_steps_per_s": round(K / (ms_dec * 1e-3), 1),
-            "gqa_decode_steps_per_s": round(K / (ms_gqa * 1e-3), 1),
-            "decode_speedup_vs_gqa": round(ms_gqa / ms_dec, 4),
-            "gva_cache_bytes": step_cache_bytes, "gqa_cache_bytes": gqa_bytes,
-            "cache_ratio": round(step_cache_bytes / gqa_bytes, 6),
-            "gqa_cache_GBs": round(gqa_bytes / (ms_gqa / K * 1e-3) / 1e9, 2),
-            "shared_kv_decode_steps_per_s": round(K / (ms_kv * 1e-3), 1),
-            "shared_kv_speedup_vs_gqa": round(ms_gqa / ms_kv, 4),
-            "shared_kv_cache_GBs": round(gqa_bytes / 2 / (ms_kv / K * 1e-3) / 1e9, 2)},
+        "gqa_comparison": gqa_cmp,
         "roofline": {"bound": "hbm",
                      "kernel": ("decode_simt_kernel" if args.fma else "decode_mma_kernel")
                                + " + combine_kernel (one gva_decode_attention call)",
-                     "achieved": round(achieved, 2), "peak": hbm_peak, "peak_kind": peak_kind,
-                     "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
-                     "alg_bytes_per_launch": alg_dec_bytes, "us_per_launch": round(dec_s * 1e6, 3),
-                     "traffic": ncu_traffic(kernel_key, wl.name)},
-        "e2e": {"value": round(job_value(step_cache_bytes, K, job_ranks, ms_e2e), 2), "unit": "GB/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(ms_e2e / K, 6), "mode": e2e_mode,
-                "serial": {"value": round(job_value(step_cache_bytes, K, job_ranks, ms_e2e_serial), 2),
-                           "ms_per_step": round(ms_e2e_serial / K, 6)}},
+                     "achieved": dec["decode_alg_GBs"], "peak": hbm_peak, "peak_kind": peak_kind,
+                     "unit": "GB/s", "frac": dec["frac_of_measured"],
+                     "alg_bytes_per_launch": st.alg_dec_bytes, "us_per_launch": dec["decode_us"],
+                     "passes": n_dec, "traffic": ncu_traffic(kernel_key, wl.name)},
+        "e2e": {"value": round(job_value(st.step_cache_bytes, 1, job_ranks, ms_e2e), 2),
+                "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(ms_e2e, 6), "mode": e2e_mode,
+                "serial": {"value": round(job_value(st.step_cache_bytes, 1, job_ranks,
+                                                    ms_e2e_serial), 2),
+                           "ms_per_step": round(ms_e2e_serial, 6)}},
         "multi_token": multi,
         "prefill": prefill,
-        "gpu_launches": (4 if split_seq else 3) * K,
+        "workloads": workloads,
+        "gpu_launches": launches_per_step * K * n_pass,
         "clocks": clocks,
     }
-    return res, di
+    return res, st.di
 
 
-def time_e2e_pipelined(step, parts, h_stage, nb, view, B, H, d_h, R, K, dev, timed):
-    """End-to-end steps with double-buffered host<->device copies.
+def time_e2e_pipelined(st, parts, h_stage, nb, view, K, dev, timer):
+    """End-to-end steps with double-buffered host<->device copies, ms per step.
 
     Step i copies its inputs (one pinned host buffer -> device staging buffer i % 2)
     on one copy stream, runs gva_decode_step on the compute stream once that copy
@@ -500,6 +677,7 @@ def time_e2e_pipelined(step, parts, h_stage, nb, view, B, H, d_h, R, K, dev, tim
     its previous copy-out has finished, so every step reads its own inputs and every
     output reaches the host."""
     NBUF = 2
+    B, H, d_h, R = st.B, st.wl.H, st.wl.d_h, st.R
     d_st = [torch.zeros(nb, dtype=torch.uint8, device=dev) for _ in range(NBUF)]
     o_dev = [torch.empty(B, H, d_h, dtype=torch.float32, device=dev) for _ in range(NBUF)]
     o_host = [torch.empty(B, H, d_h, dtype=torch.float32).pin_memory() for _ in range(NBUF)]
@@ -527,7 +705,7 @@ def time_e2e_pipelined(step, parts, h_stage, nb, view, B, H, d_h, R, K, dev, tim
                     s.wait_event(ev_in[i])
                     if i >= NBUF:
                         s.wait_event(ev_out[i - NBUF])
-                    step((first + i) % R, qq=vw[k][0], app=tuple(vw[k][1:]), o=o_dev[k])
+                    st.step((first + i) % R, qq=vw[k][0], app=tuple(vw[k][1:]), o=o_dev[k])
                     ev_done[i].record(s)
                     s_out.wait_event(ev_done[i])
                     with torch.cuda.stream(s_out):
@@ -540,61 +718,61 @@ def time_e2e_pipelined(step, parts, h_stage, nb, view, B, H, d_h, R, K, dev, tim
 
     gs, done = [], 0
     while done < K:
-        n = min(256, K - done)
+        n = min(CHUNK, K - done)
         gs.append((capture(n, done), n))
         done += n
-    for g, _ in gs:
-        g.replay()
+    timer.replay(gs)
     torch.cuda.synchronize()
-    ms, _, _ = timed(gs, K)
+    ms, _, _ = timer.timed(gs)
     # every output that reached the host equals a plain step's output (the steps
     # repeat the same inputs, and the decode is deterministic)
     o_chk = torch.empty(B, H, d_h, dtype=torch.float32, device=dev)
-    step(0, o=o_chk)
+    st.step(0, o=o_chk)
     torch.cuda.synchronize()
     for k in range(NBUF):
         assert torch.equal(o_host[k], o_chk.cpu()), "pipelined end-to-end output differs"
-    return ms
+    return ms / K
 
 
-def time_multi_token(sh, wl, di, Q, Vs, KRs, soff, slen, max_total, M, R, d, graphs_for, replay,
-                     timed, K, dev, row_bytes, part_tokens, ms_dec):
+def time_multi_token(st, Q, timer, K, dev, ms_dec):
     """Q new tokens per sequence decoded together (causal among them), as in
     speculative-decoding verification: one gva_decode_attention_multi call on the
     same caches, timed like the single-token decode."""
-    B, H, d_h, d_r = len(di.seq_len), wl.H, wl.d_h, wl.d_r
+    wl, di = st.wl, st.di
+    B, H, d_h, d_r = st.B, wl.H, wl.d_h, wl.d_r
+    d = lambda t: t.to(dev).contiguous()
     q = make_multi_queries(wl, B, Q)
     L = di.seq_len.numpy().astype(np.int64) + 1
     qpos = torch.from_numpy(np.stack([L - Q + i for i in range(Q)], 1).astype(np.int32))
     sh_q = gva.make_shape(B * Q, H, wl.G, d_h, wl.d_n, d_r, cache_dtype=wl.torch_dtype,
                           rope_base=wl.rope_base)
     q_abs = torch.empty(B, Q, H, d_h + d_r, dtype=torch.float32, device=dev)
-    gva.absorb_query(sh_q, d(q.reshape(B * Q, H, -1)), M, d(qpos.reshape(-1)), q_abs)
-    ws = torch.zeros(gva.decode_workspace_size_multi(sh, Q, max_total), dtype=torch.uint8,
+    gva.absorb_query(sh_q, d(q.reshape(B * Q, H, -1)), st.M, d(qpos.reshape(-1)), q_abs)
+    ws = torch.zeros(gva.decode_workspace_size_multi(st.sh, Q, st.max_total), dtype=torch.uint8,
                      device=dev)
     out = torch.empty(B, Q, H, d_h, dtype=torch.float32, device=dev)
 
     def call(c):
-        gva.decode_attention_multi(sh, Q, q_abs, Vs[c], KRs[c], soff, slen, max_total, out, None, ws)
+        gva.decode_attention_multi(st.sh, Q, q_abs, st.Vs[c], st.KRs[c], st.soff, st.slen,
+                                   st.max_total, out, None, ws)
 
-    for c in range(R):
+    for c in range(st.R):
         call(c)
-    gs = graphs_for(call, K)
-    replay(gs)
-    ms, _, _ = timed(gs, K)
+    ms, _, _ = timer.time_fn(call, K, st.R)
     assert gva.workspace_status(ws) == 0, "device status word set"
-    s = ms / K * 1e-3
-    alg = part_tokens * row_bytes + B * Q * H * (d_h + d_r) * 4 + B * Q * H * d_h * 4
+    s = ms * 1e-3
+    alg = st.part_tokens * st.row_bytes + B * Q * H * (d_h + d_r) * 4 + B * Q * H * d_h * 4
     return {"n_query": Q, "call": "gva_decode_attention_multi", "us_per_call": round(s * 1e6, 3),
             "alg_GBs": round(alg / s / 1e9, 2), "time_vs_single_token_decode": round(ms / ms_dec, 4)}
 
 
-def time_prefill(wl, di, Q, graphs_for, replay, timed, d, dev, steps):
+def time_prefill(wl, di, Q, timer, dev, steps):
     """Chunked prefill: Q new tokens appended to every sequence of the batch
     (positions L .. L+Q-1, causal among them), one gva_decode_attention_multi
-    call on the tcgen05 kernel.  Returns the call time and its algorithmic
+    call on the tcgen05 kernel.  Returns the call time (ms) and its algorithmic
     tensor work: per (query row, visible key) 2*(2*d_h + d_r) flops, the scores
     q~.v + q_r.k_rope and the output p*v."""
+    d = lambda t: t.to(dev).contiguous()
     L = di.seq_len.numpy().astype(np.int64) + Q
     B, H = len(L), wl.H
     dq = make_decode_inputs(wl, extra_slots=0, lengths=L)
@@ -608,7 +786,7 @@ def time_prefill(wl, di, Q, graphs_for, replay, timed, d, dev, steps):
                         rope_base=wl.rope_base)
     tot = int(L.sum())
     cb = dq.V.numel() * dq.V.element_size() + dq.k_rope.numel() * dq.k_rope.element_size()
-    R = max(2, math.ceil(3 * L2_BYTES / cb))
+    R = copies_for(cb)
     Vs = [d(dq.V) for _ in range(R)]
     Ks = [d(dq.k_rope) for _ in range(R)]
     soff, slen = d(dq.seq_offset), d(dq.seq_len)
@@ -616,61 +794,16 @@ def time_prefill(wl, di, Q, graphs_for, replay, timed, d, dev, steps):
     out = torch.empty(B, Q, H, wl.d_h, dtype=torch.float32, device=dev)
 
     def call(c):
-        c %= R   # graphs_for counts copies of the step's cache
         gva.decode_attention_multi(sh, Q, q_abs, Vs[c], Ks[c], soff, slen, tot, out, None, ws)
 
     for c in range(R):
         call(c)
     n = max(10, min(steps, 200))
-    gs = graphs_for(call, n)
-    replay(gs)
-    ms, _, _ = timed(gs, n)
+    ms, _, _ = timer.time_fn(call, n, R)
     assert gva.workspace_status(ws) == 0, "device status word set"
     keys = int(sum(Q * (int(l) - Q) + Q * (Q + 1) // 2 for l in L))
     flops = keys * H * 2 * (2 * wl.d_h + wl.d_r)
-    return ms / n, flops
-
-
-def run_gqa_comparison(args, wl, B, H, G, d_h, R, flags, d, graphs_for, replay, timed, dev):
-    """Same-shape GQA decode (K and V cache) timed like the GVA decode."""
-    gi = make_gqa_inputs(wl, extra_slots=1)
-    Kq = [d(gi.K) for _ in range(R)]
-    Vq = [d(gi.V) for _ in range(R)]
-    sh_q = gva.make_shape(B, H, G, d_h, d_h, 0, cache_dtype=wl.torch_dtype, flags=flags,
-                          ctas_per_sm=args.ctas_per_sm)
-    qg = d(gi.q)
-    slen_q = d(torch.from_numpy((gi.seq_len.numpy() + 1).astype(np.int32)))
-    soff_q = d(gi.seq_offset)
-    tot_q = int(gi.seq_len.numpy().astype(np.int64).sum()) + B
-    ws_q = gva.new_workspace(sh_q, tot_q, device=dev)
-    out_q = torch.empty(B, H, d_h, dtype=torch.float32, device=dev)
-
-    def gqa_decode(c):
-        gva.gqa_decode_attention(sh_q, qg, Kq[c], Vq[c], soff_q, slen_q, tot_q, out_q, None, ws_q)
-
-    for c in range(R):
-        gqa_decode(c)
-    g_gqa = graphs_for(gqa_decode, args.steps)
-    replay(g_gqa)
-    ms_gqa, _, _ = timed(g_gqa, args.steps)
-    del g_gqa
-
-    # shared keys and values (K = V, the pages' first design): the same batch
-    # with the value cache only, through gva_shared_kv_decode_attention
-    sh_kv = gva.make_shape(B, H, G, d_h, d_h, 0, cache_dtype=wl.torch_dtype, flags=flags,
-                           ctas_per_sm=args.ctas_per_sm)
-    ws_kv = gva.new_workspace(sh_kv, tot_q, device=dev)
-
-    def kv_decode(c):
-        gva.shared_kv_decode_attention(sh_kv, qg, Vq[c], soff_q, slen_q, tot_q, out_q, None, ws_kv)
-
-    for c in range(R):
-        kv_decode(c)
-    g_kv = graphs_for(kv_decode, args.steps)
-    replay(g_kv)
-    ms_kv, _, _ = timed(g_kv, args.steps)
-    assert gva.workspace_status(ws_kv) == 0, "device status word set"
-    return ms_gqa, tot_q * 2 * G * d_h * wl.elem_bytes, ms_kv
+    return ms, flops
 
 
 # ----------------------------------------------------------------------------- oracle arm
@@ -686,7 +819,7 @@ def oracle_threads():
 
 def time_oracle(wl, di, budget_s, max_units=None):
     """Oracle decode on (sequence, head) pairs until the time budget is spent.
-    Returns (cache bytes attended per second, description)."""
+    Returns (cache bytes attended per second, description, seconds, pairs)."""
     import oracle
     from compressed_kv_cache_gva_b200.synth import as_f64
     q, M = as_f64(di.q), as_f64(di.M)

@@ -10,6 +10,7 @@ from __future__ import annotations
 
 import concurrent.futures as cf
 import glob
+import hashlib
 import os
 import subprocess
 import sys
@@ -36,22 +37,29 @@ def _deps():
             + glob.glob(os.path.join(INCLUDE, "*.h")) + [os.path.abspath(__file__)])
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+# Test-only variant for the failure-detection test: bounded pipeline waits give up
+# after 50 ms, and the split kernel's producer never requests the second tile of
+# each CTA, so a consumer wait runs out (no copy is ever in flight for that tile).
+WAIT_TEST_LIB = os.path.join(PKG, "libgva_waittest.so")
+WAIT_TEST_FLAGS = ("-DGVA_WAIT_NS=50000000ull", "-DGVA_TEST_WITHHOLD_TILE=1")
+
+
+def up_to_date(out: str = LIB) -> bool:
+    if not os.path.exists(out):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(out)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
 def build(force: bool = False, verbose: bool = False, extra_flags=(), out: str = LIB) -> str:
     """Compile every csrc/*.cu and link them into `out` (default: the package's
     libgva.so).  `extra_flags` go to every nvcc compile (e.g. -DGVA_TRACE)."""
-    if not force and not extra_flags and out == LIB and up_to_date():
-        return LIB
+    if not force and up_to_date(out) and (not extra_flags or out != LIB):
+        return out
     os.makedirs(OBJDIR, exist_ok=True)
     srcs = _sources()
 
-    tag = "" if not extra_flags else "_" + str(abs(hash(tuple(extra_flags))))
+    tag = "" if not extra_flags else "_" + hashlib.sha1(" ".join(extra_flags).encode()).hexdigest()[:12]
     def compile_one(src):
         obj = os.path.join(OBJDIR, os.path.basename(src) + tag + ".o")
         cmd = [NVCC, *FLAGS, *extra_flags, "-c", src, "-o", obj]
@@ -72,6 +80,11 @@ def build(force: bool = False, verbose: bool = False, extra_flags=(), out: str =
         raise RuntimeError(f"link failed:\n{r.stderr}")
     os.replace(tmp, out)
     return out
+
+
+def build_wait_test(force: bool = False) -> str:
+    """The failure-detection test's library (see WAIT_TEST_FLAGS)."""
+    return build(force=force, extra_flags=WAIT_TEST_FLAGS, out=WAIT_TEST_LIB)
 
 
 if __name__ == "__main__":

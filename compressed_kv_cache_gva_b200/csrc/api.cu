@@ -146,7 +146,8 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
                            const int32_t* seq_len, int64_t max_total_tokens, int64_t num_slots,
                            void* out, float* lse, void* workspace, size_t ws_bytes, void* stream,
                            bool prefetch = false, const int32_t* new_slots = nullptr,
-                           int n_new = 0, int nq = 1, bool raw_q = false) {
+                           int n_new = 0, int nq = 1, bool raw_q = false,
+                           bool clear_status = false) {
   gva_status_t s = check_shape(shp, gqa);
   if (s != GVA_OK) return s;
   if (nq < 1 || nq > 64) return fail(GVA_ERR_INVALID_ARG, "n_query=%d outside [1,64]", nq);
@@ -209,6 +210,11 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
   a.trace = g_trace;
 #endif
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // clear_status: zero the workspace's status word on the stream right before the
+  // split kernel, once every check has passed (a rejected call enqueues nothing)
+  auto clear = [&]() -> cudaError_t {
+    return clear_status ? cudaMemsetAsync(a.status, 0, sizeof(int), st) : cudaSuccess;
+  };
 
   cudaError_t err;
   if (p.tc) {
@@ -225,6 +231,7 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
                          drp == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B)) != GVA_OK)
         return s;
     }
+    if ((err = clear()) != cudaSuccess) return cuda_fail(err, "clearing the status word");
     err = gva::launch_decode_tc(sh, a, tv, tk, st);
   } else if (p.mma) {
     a.tile = gva::mma_tile(sh, gqa);
@@ -242,9 +249,14 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
                          drp == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B)) != GVA_OK)
         return s;
     }
+    if ((err = clear()) != cudaSuccess) return cuda_fail(err, "clearing the status word");
     err = gva::launch_decode_mma(sh, gqa, a, tx, tv, tk, st);
   } else {
     a.tile = gva::simt_tile();
+    if (!gva::simt_supported(sh, gqa))
+      return fail(GVA_ERR_UNSUPPORTED, "no decode kernel for H=%d G=%d d_h=%d d_r=%d", sh.H, sh.G,
+                  sh.d_h, sh.d_r);
+    if ((err = clear()) != cudaSuccess) return cuda_fail(err, "clearing the status word");
     err = gva::launch_decode_simt(sh, gqa, a, st);
     if (err == cudaErrorNotSupported)
       return fail(GVA_ERR_UNSUPPORTED, "no decode kernel for H=%d G=%d d_h=%d d_r=%d", sh.H, sh.G,
@@ -262,6 +274,20 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
 namespace gva {
 // Lets other translation units of the library record a reason for gva_last_error.
 void set_error_message(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+
+// gva_decode_attention that also zeroes the workspace's status word on the stream,
+// after validation and right before the split kernel (used by the entry point
+// whose scratch is shared by all calls).
+gva_status_t decode_attention_clearing_status(const gva_shape_t* shape, const float* q_abs,
+                                              const void* V_cache, const void* kr_cache,
+                                              const int32_t* seq_offset, const int32_t* seq_len,
+                                              int64_t max_total_tokens, int64_t num_slots,
+                                              void* out, float* lse, void* workspace,
+                                              size_t ws_bytes, void* stream) {
+  return decode_common(shape, false, q_abs, V_cache, V_cache, kr_cache, seq_offset, seq_len,
+                       max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream, false,
+                       nullptr, 0, 1, false, /*clear_status=*/true);
+}
 }  // namespace gva
 
 extern "C" {
@@ -517,6 +543,83 @@ gva_status_t gva_merge_states(const gva_shape_t* shape, int32_t R, const float* 
   cudaError_t e = gva::launch_merge_states(*shape, R, outs, lses, out, lse,
                                            static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? GVA_OK : cuda_fail(e, "merge launch");
+}
+
+// Argument checks of the GQA append and query rotation (shape checked as GQA).
+static gva_status_t gqa_rope_check(const gva_shape_t& sh) {
+  if (sh.d_h % 2 || sh.d_h > 2 * gva::kMaxRopePairs)
+    return fail(GVA_ERR_UNSUPPORTED, "GQA RoPE needs an even d_h <= %d (d_h=%d)",
+                2 * gva::kMaxRopePairs, sh.d_h);
+  if (!(sh.rope_base > 0.0) || !isfinite(sh.rope_base))
+    return fail(GVA_ERR_INVALID_ARG, "rope_base must be positive and finite");
+  if ((sh.G * sh.d_h * elt(sh.cache_dtype)) % 16)
+    return fail(GVA_ERR_INVALID_ARG, "cache rows must be multiples of 16 bytes");
+  return GVA_OK;
+}
+
+static gva_status_t gqa_append_check(const gva_shape_t& sh, const void* k_new, const void* v_new,
+                                     const int32_t* slot, const int32_t* pos, int64_t num_slots,
+                                     const void* K_cache, const void* V_cache) {
+  if (!k_new || !v_new || !slot || !pos || !K_cache || !V_cache)
+    return fail(GVA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(slot) || !aligned16(pos) ||
+      !aligned16(K_cache) || !aligned16(V_cache))
+    return fail(GVA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (num_slots < 1) return fail(GVA_ERR_INVALID_ARG, "num_slots=%lld < 1", (long long)num_slots);
+  return GVA_OK;
+}
+
+gva_status_t gqa_append_cache(const gva_shape_t* shape, int32_t N, const void* k_new,
+                              const void* v_new, const int32_t* slot, const int32_t* pos,
+                              int64_t num_slots, void* K_cache, void* V_cache, int32_t* err_flag,
+                              void* stream) {
+  gva_status_t s = check_shape(shape, true);
+  if (s != GVA_OK) return s;
+  if ((s = gqa_rope_check(*shape)) != GVA_OK) return s;
+  if (N < 0) return fail(GVA_ERR_INVALID_ARG, "N=%d < 0", N);
+  if (N == 0) return GVA_OK;
+  if ((s = gqa_append_check(*shape, k_new, v_new, slot, pos, num_slots, K_cache, V_cache)) != GVA_OK)
+    return s;
+  cudaError_t e = gva::launch_gqa_append(*shape, N, k_new, v_new, slot, pos, num_slots, K_cache,
+                                         V_cache, err_flag, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GVA_OK : cuda_fail(e, "GQA append launch");
+}
+
+gva_status_t gqa_decode_step(const gva_shape_t* shape, const void* q, const int32_t* q_pos,
+                             int32_t n_new, const void* k_new, const void* v_new,
+                             const int32_t* slot, const int32_t* pos, void* K_cache,
+                             void* V_cache, int64_t num_slots, const int32_t* seq_offset,
+                             const int32_t* seq_len, int64_t max_total_tokens, float* q_rot,
+                             void* out, float* lse, int32_t* err_flag, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  gva_status_t s = check_shape(shape, true);
+  if (s != GVA_OK) return s;
+  if ((s = gqa_rope_check(*shape)) != GVA_OK) return s;
+  if (n_new < 0) return fail(GVA_ERR_INVALID_ARG, "n_new=%d < 0", n_new);
+  if (shape->B == 0 && n_new == 0) return GVA_OK;
+  if (!q_rot || !q || !q_pos || !K_cache || !V_cache || !seq_offset || !seq_len || !out ||
+      !workspace)
+    return fail(GVA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned16(q) || !aligned16(q_pos) || !aligned16(q_rot))
+    return fail(GVA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (n_new > 0 &&
+      (s = gqa_append_check(*shape, k_new, v_new, slot, pos, num_slots, K_cache, V_cache)) != GVA_OK)
+    return s;
+  // the decode reads the rotated float32 query
+  gva_shape_t shd = *shape;
+  shd.q_dtype = GVA_F32;
+  Plan p;
+  if ((s = plan_decode(shd, true, max_total_tokens, &p, false)) != GVA_OK) return s;
+  if (ws_bytes < p.ws.total)
+    return fail(GVA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, p.ws.total);
+  cudaError_t e = gva::launch_gqa_prep(*shape, q, q_pos, q_rot, n_new, k_new, v_new, slot, pos,
+                                       num_slots, K_cache, V_cache, err_flag,
+                                       static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "GQA query rotation + append launch");
+  if (shape->B == 0) return GVA_OK;
+  return decode_common(&shd, true, q_rot, K_cache, V_cache, nullptr, seq_offset, seq_len,
+                       max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream,
+                       /*prefetch=*/true, slot, n_new);
 }
 
 gva_status_t gqa_decode_attention(const gva_shape_t* shape, const void* q, const void* K_cache,

@@ -18,7 +18,18 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kMaxBatch = 4096;          // sequences per call (prefix array lives in smem)
 constexpr int kMaxQueryRows = 65535 * 4; // query rows of one absorb call (its grid's y extent)
-constexpr uint32_t kWaitLimit = 1u << 22;  // iterations of a bounded mbarrier wait
+// A bounded mbarrier wait gives up after GVA_WAIT_LIMIT polls or GVA_WAIT_NS
+// nanoseconds of %globaltimer, whichever comes first.  The time bound makes the
+// worst case independent of how long one poll blocks; the failure-detection test
+// build shortens it.
+#ifndef GVA_WAIT_LIMIT
+#define GVA_WAIT_LIMIT (1u << 22)
+#endif
+#ifndef GVA_WAIT_NS
+#define GVA_WAIT_NS 2000000000ull
+#endif
+constexpr uint32_t kWaitLimit = GVA_WAIT_LIMIT;
+constexpr unsigned long long kWaitNs = GVA_WAIT_NS;
 
 // ---------------------------------------------------------------------------
 // Workspace: [status word | meta[B] | partial (m,l)[P][H] | partial o[P][H][d_h]]
@@ -383,10 +394,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait: gives up after kWaitLimit polls and reports it in the status word.
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait: gives up after kWaitLimit polls or kWaitNs nanoseconds and reports
+// it in the status word.  The clock is read only once the first poll has failed,
+// and then every 64 polls.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* status) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i)
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t i = 1; i < kWaitLimit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63) == 0 && global_ns() - t0 > kWaitNs) break;
+  }
   atomicOr(status, GVA_DEVERR_WAIT);
   return false;
 }

@@ -152,6 +152,12 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
   auto issue = [&](int k) {
     const int s = k % C::STAGES;
     const uint32_t fb = smem_u32(full + s);
+#ifdef GVA_TEST_WITHHOLD_TILE
+    // Failure-detection test builds only: this tile ordinal of every CTA is never
+    // requested (no transaction is armed and no copy is in flight for it), so the
+    // consumers' bounded wait on its barrier runs out and reports GVA_DEVERR_WAIT.
+    if (k == GVA_TEST_WITHHOLD_TILE) return;
+#endif
     if (k == 0) trace_mark(a, 2);
     trace_tile(a, k, 0);
     mbar_arrive_expect_tx(fb, C::TX);

@@ -187,6 +187,8 @@ static bool simt_ok(const gva_shape_t& sh, bool gqa) {
          simt_layout(sh, gqa).total <= 200 * 1024;
 }
 
+bool simt_supported(const gva_shape_t& sh, bool gqa) { return simt_ok(sh, gqa); }
+
 int simt_grid(const gva_shape_t& sh, int num_sms, long long max_total_tokens, bool gqa) {
   const size_t smem = simt_layout(sh, gqa).total;
   int per_sm = (int)((220 * 1024) / (smem + 1024));
@@ -203,7 +205,7 @@ cudaError_t launch_decode_simt(const gva_shape_t& sh, bool gqa, DecodeArgs& a, c
   const SimtLayout Ly = simt_layout(sh, gqa);
   auto k = sh.cache_dtype == GVA_BF16 ? decode_simt_kernel<__nv_bfloat16> : decode_simt_kernel<float>;
   if (Ly.total > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Ly.total);
+    cudaError_t e = ensure_max_smem(k, Ly.total);
     if (e != cudaSuccess) return e;
   }
   return launch_pdl(k, dim3(a.grid), dim3(kSimtThreads), Ly.total, st, a, Ly, gqa ? 1 : 0);

@@ -690,7 +690,7 @@ cudaError_t run_tc(const gva_shape_t& sh, DecodeArgs& a, const CUtensorMap& tv,
                    const CUtensorMap& tk, cudaStream_t st) {
   const size_t smem = C::smem_bytes(sh.B);
   auto k = decode_tc_kernel<C>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_max_smem(k, smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(k, dim3(a.grid), dim3(C::THREADS), smem, st, a, tv, tk);
 }

@@ -13,14 +13,36 @@ namespace gva {
 
 struct DecodeArgs;
 
+// Function attributes already applied on the current device (launch.cu): a
+// launcher sets an attribute only when attr_applied() says the device has not
+// yet received that value (or a larger one) for the kernel.
+bool attr_applied(const void* kernel, int attr, long long value);
+void attr_record(const void* kernel, int attr, long long value);
+
+// Raise a kernel's dynamic shared-memory limit to at least `smem` bytes, once
+// per kernel, device and size.
+template <typename... KArgs>
+cudaError_t ensure_max_smem(void (*k)(KArgs...), size_t smem) {
+  const void* key = reinterpret_cast<const void*>(k);
+  const int attr = (int)cudaFuncAttributeMaxDynamicSharedMemorySize;
+  if (attr_applied(key, attr, (long long)smem)) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess) attr_record(key, attr, (long long)smem);
+  return e;
+}
+
 // Launch with programmatic stream serialization allowed (see pdl_wait).
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                        Args&&... args) {
-  // Every kernel asks for the maximum shared-memory carveout, so consecutive
-  // kernels never force the SM to reconfigure its L1/shared split in between.
-  cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
-                       (int)cudaSharedmemCarveoutMaxShared);
+  // Every kernel asks for the maximum shared-memory carveout (once per device), so
+  // consecutive kernels never force the SM to reconfigure its L1/shared split.
+  const void* key = reinterpret_cast<const void*>(k);
+  const int carve = (int)cudaFuncAttributePreferredSharedMemoryCarveout;
+  if (!attr_applied(key, carve, 1) &&
+      cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared) == cudaSuccess)
+    attr_record(key, carve, 1);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -51,6 +73,17 @@ cudaError_t launch_prep_step(const gva_shape_t& sh, const void* q, const void* M
                              const int* slot, const int* pos, long long num_slots, void* V_cache,
                              void* kr_cache, int* err_flag, cudaStream_t st);
 
+// Same-shape GQA: append (key rotated over d_h, value copied) and the first
+// kernel of its decode step (query rotation + append; the next kernel may launch
+// at once).
+cudaError_t launch_gqa_append(const gva_shape_t& sh, int N, const void* k_new, const void* v_new,
+                              const int* slot, const int* pos, long long num_slots, void* K_cache,
+                              void* V_cache, int* err_flag, cudaStream_t st);
+cudaError_t launch_gqa_prep(const gva_shape_t& sh, const void* q, const int* q_pos, float* q_rot,
+                            int N, const void* k_new, const void* v_new, const int* slot,
+                            const int* pos, long long num_slots, void* K_cache, void* V_cache,
+                            int* err_flag, cudaStream_t st);
+
 // Multi-token attention on tcgen05 (prefill_tc.cu): nq new tokens per sequence,
 // causal among them, rows = tokens x heads of a group in blocks of 128.  The
 // value tensor map's box is prefill_tile_rows(sh) x 64, the k_rope map's
@@ -64,6 +97,7 @@ cudaError_t launch_prefill(const gva_shape_t& sh, int nq, const float* q_abs,
 
 // CUDA-core split kernel (any dtype / shape within limits).  Returns
 // cudaErrorNotSupported for shapes it is not built for.
+bool simt_supported(const gva_shape_t& sh, bool gqa);
 int simt_grid(const gva_shape_t& sh, int num_sms, long long max_total_tokens, bool gqa);
 int simt_tile();
 cudaError_t launch_decode_simt(const gva_shape_t& sh, bool gqa, DecodeArgs& a, cudaStream_t st);

@@ -11,6 +11,12 @@
 
 namespace gva {
 void set_error_message(const char* msg);   // defined in api.cu
+gva_status_t decode_attention_clearing_status(const gva_shape_t* shape, const float* q_abs,
+                                              const void* V_cache, const void* kr_cache,
+                                              const int32_t* seq_offset, const int32_t* seq_len,
+                                              int64_t max_total_tokens, int64_t num_slots,
+                                              void* out, float* lse, void* workspace,
+                                              size_t ws_bytes, void* stream);   // api.cu
 }
 
 namespace {
@@ -66,15 +72,30 @@ extern "C" gva_status_t gva_decode_attention_noalloc(const gva_shape_t* shape, c
   }
   void* ws = scratch_address();
   if (!ws) return GVA_ERR_CUDA;
-  // the previous call's device status word must not leak into this one
-  const cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int), static_cast<cudaStream_t>(stream));
+  // The previous call's device status word must not leak into this one: the
+  // decode zeroes it on the stream after all its checks have passed, so a call
+  // rejected on the host writes nothing into the shared scratch.
+  return gva::decode_attention_clearing_status(shape, q_abs, V_cache, kr_cache, seq_offset, seq_len,
+                                               max_total_tokens, num_slots, out, lse, ws,
+                                               (size_t)GVA_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+extern "C" gva_status_t gva_noalloc_status(int32_t* status_out, void* stream) {
+  if (!status_out) {
+    gva::set_error_message("status_out is NULL");
+    return GVA_ERR_INVALID_ARG;
+  }
+  void* ws = scratch_address();
+  if (!ws) return GVA_ERR_CUDA;
+  // the status word is the first int32 of the scratch (the workspace layout)
+  const cudaError_t e = cudaMemcpyAsync(status_out, ws, sizeof(int32_t), cudaMemcpyDefault,
+                                        static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     char msg[200];
-    snprintf(msg, sizeof(msg), "clearing the static scratch status word failed: %s",
+    snprintf(msg, sizeof(msg), "copying the static scratch status word failed: %s",
              cudaGetErrorString(e));
     gva::set_error_message(msg);
     return GVA_ERR_CUDA;
   }
-  return gva_decode_attention(shape, q_abs, V_cache, kr_cache, seq_offset, seq_len, max_total_tokens,
-                              num_slots, out, lse, ws, (size_t)GVA_NOALLOC_SCRATCH_BYTES, stream);
+  return GVA_OK;
 }

@@ -433,7 +433,7 @@ template <class C>
 cudaError_t run_prefill(const PrefillArgs& a, const CUtensorMap& tv, const CUtensorMap& tk,
                         cudaStream_t st) {
   auto k = prefill_tc_kernel<C>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  cudaError_t e = ensure_max_smem(k, (size_t)C::SMEM);
   if (e != cudaSuccess) return e;
   const int nblk = (a.nq * a.hpr + C::M - 1) / C::M;
   return launch_pdl(k, dim3(nblk, a.G, a.B), dim3(C::THREADS), C::SMEM, st, a, tv, tk);

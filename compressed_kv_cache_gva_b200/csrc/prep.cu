@@ -259,6 +259,223 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Same-shape GQA: the matched baseline caches a key AND a value per group and
+// token (onedev.kr review, "What differs": N_GQA = 2*T*G*d_h).  Its keys carry
+// RoPE over the whole head width, pair (i, i + d_h/2) rotated by
+// pos * base^(-2i/d_h); the key is stored rounded once to the cache type and the
+// value unchanged.  The query of a step is rotated the same way (float32 out,
+// unscaled: the decode kernel applies softmax_scale).
+// ---------------------------------------------------------------------------
+
+// One warp per new token: the value row and the key pairs are loaded and the
+// rotation computed (one float64 sincos per pair index, shared by the groups)
+// before waiting on the preceding kernel; the stores come after.
+constexpr int kGqaMaxGroups = 8;   // key pairs of up to this many groups held in registers
+template <typename T>
+__device__ __forceinline__ void gqa_append_block(long long bx, int N, int G, int d_h,
+                                                 const T* __restrict__ k_new,
+                                                 const T* __restrict__ v_new,
+                                                 const int* __restrict__ slot,
+                                                 const int* __restrict__ pos, long long num_slots,
+                                                 T* __restrict__ K_cache, T* __restrict__ V_cache,
+                                                 int* __restrict__ err_flag, const RopeTable& rt,
+                                                 int early_trigger) {
+  constexpr int kVecPerLane = 4;   // value rows up to 2 KB in registers
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long i = bx * warps + (threadIdx.x >> 5);
+  const bool active = i < N;
+  const long long s = active ? slot[i] : -1;
+  const bool ok = active && s >= 0 && s < num_slots;
+  const int row = G * d_h, half = d_h / 2;
+  const int nvec = row * (int)sizeof(T) / 16;
+  const uint4* vs = reinterpret_cast<const uint4*>(v_new + (ok ? i : 0) * row);
+  uint4 r[kVecPerLane];
+#pragma unroll
+  for (int u = 0; u < kVecPerLane; ++u)
+    if (ok && lane + 32 * u < nvec) r[u] = vs[lane + 32 * u];
+  const T* krow = k_new + (ok ? i : 0) * row;
+  const bool kreg = G <= kGqaMaxGroups;
+  float kx[kGqaMaxGroups][2][2];   // [group][pair index u][x1, x2]
+#pragma unroll
+  for (int g = 0; g < kGqaMaxGroups; ++g)
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int k = lane + 32 * u;
+      const bool on = ok && kreg && g < G && k < half;
+      kx[g][u][0] = on ? to_f32(krow[g * d_h + k]) : 0.f;
+      kx[g][u][1] = on ? to_f32(krow[g * d_h + half + k]) : 0.f;
+    }
+  double cs[2] = {1.0, 1.0}, sn[2] = {0.0, 0.0};   // d_h <= 128: two pair indices per lane
+  if (ok) {
+    const double p = (double)pos[i];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int k = lane + 32 * u;
+      if (k < half) sincos(p * rt.inv_freq[k], &sn[u], &cs[u]);
+    }
+  }
+  pdl_wait();
+  if (!early_trigger) pdl_trigger();
+  if (active && !ok) {
+    if (lane == 0 && err_flag) atomicExch(err_flag, 1);
+    return;
+  }
+  if (!ok) return;
+  // value: bit-exact copy
+  uint4* vd = reinterpret_cast<uint4*>(V_cache + s * row);
+#pragma unroll
+  for (int u = 0; u < kVecPerLane; ++u)
+    if (lane + 32 * u < nvec) vd[lane + 32 * u] = r[u];
+  for (int e = lane + 32 * kVecPerLane; e < nvec; e += 32) vd[e] = vs[e];   // wider rows
+  // key: every group's pairs rotated, rounded once
+  T* kd = K_cache + s * row;
+  auto put = [&](int g, int u, double x1, double x2) {
+    const int k = lane + 32 * u;
+    store_rounded(kd + g * d_h + k, x1 * cs[u] - x2 * sn[u]);
+    store_rounded(kd + g * d_h + half + k, x1 * sn[u] + x2 * cs[u]);
+  };
+  if (kreg) {
+#pragma unroll
+    for (int g = 0; g < kGqaMaxGroups; ++g)
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+        if (g < G && lane + 32 * u < half) put(g, u, kx[g][u][0], kx[g][u][1]);
+  } else {
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int k = lane + 32 * u;
+        if (k < half) put(g, u, to_f32(krow[g * d_h + k]), to_f32(krow[g * d_h + half + k]));
+      }
+  }
+}
+
+// One warp per (sequence, head) row of the query: q_rot = RoPE(q, q_pos[b])
+// over d_h, float32.
+template <typename TQ>
+__device__ __forceinline__ void gqa_qrot_block(long long bx, int rows, int H, int d_h,
+                                               const TQ* __restrict__ q,
+                                               const int* __restrict__ q_pos,
+                                               float* __restrict__ q_rot, const RopeTable& rt,
+                                               int early_trigger) {
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long r = bx * warps + (threadIdx.x >> 5);
+  const bool active = r < rows;
+  const int half = d_h / 2;
+  double y1[2] = {0.0, 0.0}, y2[2] = {0.0, 0.0};
+  if (active) {
+    const double p = (double)q_pos[r / H];
+    const TQ* qr = q + r * d_h;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int k = lane + 32 * u;
+      if (k < half)
+        rope_pair((double)to_f32(qr[k]), (double)to_f32(qr[half + k]), p, rt.inv_freq[k], y1[u],
+                  y2[u]);
+    }
+  }
+  pdl_wait();
+  if (!early_trigger) pdl_trigger();
+  if (!active) return;
+  float* o = q_rot + r * d_h;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int k = lane + 32 * u;
+    if (k < half) {
+      o[k] = (float)y1[u];
+      o[half + k] = (float)y2[u];
+    }
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+    gqa_append_kernel(int N, int G, int d_h, const T* __restrict__ k_new,
+                      const T* __restrict__ v_new, const int* __restrict__ slot,
+                      const int* __restrict__ pos, long long num_slots, T* __restrict__ K_cache,
+                      T* __restrict__ V_cache, int* __restrict__ err_flag, const RopeTable rt) {
+  gqa_append_block<T>(blockIdx.x, N, G, d_h, k_new, v_new, slot, pos, num_slots, K_cache, V_cache,
+                      err_flag, rt, 0);
+}
+
+// The first kernel of the GQA decode step, the counterpart of prep_step_kernel:
+// blocks [0, n_qrot) rotate the queries (8 rows per block), the rest append the
+// new tokens (8 per block).  The successor may launch at once (see
+// prep_step_kernel).
+template <typename TQ, typename T>
+__global__ void __launch_bounds__(256)
+    gqa_prep_kernel(int n_qrot, int rows, int H, int d_h, const TQ* __restrict__ q,
+                    const int* __restrict__ q_pos, float* __restrict__ q_rot, int N, int G,
+                    const T* __restrict__ k_new, const T* __restrict__ v_new,
+                    const int* __restrict__ slot, const int* __restrict__ pos, long long num_slots,
+                    T* __restrict__ K_cache, T* __restrict__ V_cache, int* __restrict__ err_flag,
+                    const RopeTable rt) {
+  pdl_trigger();
+  if ((int)blockIdx.x < n_qrot)
+    gqa_qrot_block<TQ>(blockIdx.x, rows, H, d_h, q, q_pos, q_rot, rt, 1);
+  else
+    gqa_append_block<T>(blockIdx.x - n_qrot, N, G, d_h, k_new, v_new, slot, pos, num_slots,
+                        K_cache, V_cache, err_flag, rt, 1);
+}
+
+static RopeTable rope_table_width(double base, int width) {
+  RopeTable t{};
+  for (int i = 0; i < width / 2 && i < kMaxRopePairs; ++i)
+    t.inv_freq[i] = pow(base, -2.0 * (double)i / (double)width);
+  return t;
+}
+
+cudaError_t launch_gqa_append(const gva_shape_t& sh, int N, const void* k_new, const void* v_new,
+                              const int* slot, const int* pos, long long num_slots, void* K_cache,
+                              void* V_cache, int* err_flag, cudaStream_t st) {
+  const int grid = (int)(((long long)N + 7) / 8);
+  const RopeTable rt = rope_table_width(sh.rope_base, sh.d_h);
+  if (sh.cache_dtype == GVA_BF16)
+    return launch_pdl(gqa_append_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, N, sh.G,
+                      sh.d_h, (const __nv_bfloat16*)k_new, (const __nv_bfloat16*)v_new, slot, pos,
+                      num_slots, (__nv_bfloat16*)K_cache, (__nv_bfloat16*)V_cache, err_flag, rt);
+  return launch_pdl(gqa_append_kernel<float>, dim3(grid), dim3(256), 0, st, N, sh.G, sh.d_h,
+                    (const float*)k_new, (const float*)v_new, slot, pos, num_slots,
+                    (float*)K_cache, (float*)V_cache, err_flag, rt);
+}
+
+template <typename TQ, typename T>
+static cudaError_t launch_gqa_prep_t(const gva_shape_t& sh, const void* q, const int* q_pos,
+                                     float* q_rot, int N, const void* k_new, const void* v_new,
+                                     const int* slot, const int* pos, long long num_slots,
+                                     void* K_cache, void* V_cache, int* err_flag,
+                                     cudaStream_t st) {
+  const long long rows = (long long)sh.B * sh.H;
+  const long long n_qrot = (rows + 7) / 8, n_app = ((long long)N + 7) / 8;
+  if (n_qrot + n_app > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  return launch_pdl(gqa_prep_kernel<TQ, T>, dim3((unsigned)(n_qrot + n_app)), dim3(256), 0, st,
+                    (int)n_qrot, (int)rows, sh.H, sh.d_h, (const TQ*)q, q_pos, q_rot, N, sh.G,
+                    (const T*)k_new, (const T*)v_new, slot, pos, num_slots, (T*)K_cache,
+                    (T*)V_cache, err_flag, rope_table_width(sh.rope_base, sh.d_h));
+}
+
+cudaError_t launch_gqa_prep(const gva_shape_t& sh, const void* q, const int* q_pos, float* q_rot,
+                            int N, const void* k_new, const void* v_new, const int* slot,
+                            const int* pos, long long num_slots, void* K_cache, void* V_cache,
+                            int* err_flag, cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  const bool qb = sh.q_dtype == GVA_BF16, cb = sh.cache_dtype == GVA_BF16;
+  if (qb && cb)
+    return launch_gqa_prep_t<bf, bf>(sh, q, q_pos, q_rot, N, k_new, v_new, slot, pos, num_slots,
+                                     K_cache, V_cache, err_flag, st);
+  if (qb)
+    return launch_gqa_prep_t<bf, float>(sh, q, q_pos, q_rot, N, k_new, v_new, slot, pos,
+                                        num_slots, K_cache, V_cache, err_flag, st);
+  if (cb)
+    return launch_gqa_prep_t<float, bf>(sh, q, q_pos, q_rot, N, k_new, v_new, slot, pos,
+                                        num_slots, K_cache, V_cache, err_flag, st);
+  return launch_gqa_prep_t<float, float>(sh, q, q_pos, q_rot, N, k_new, v_new, slot, pos,
+                                         num_slots, K_cache, V_cache, err_flag, st);
+}
+
 static RopeTable rope_table(const gva_shape_t& sh) {
   RopeTable t{};
   for (int i = 0; i < sh.d_r / 2 && i < kMaxRopePairs; ++i)
@@ -278,13 +495,13 @@ cudaError_t launch_absorb(const gva_shape_t& sh, const void* q, const void* M, c
   const RopeTable rt = rope_table(sh);
   if (sh.q_dtype == GVA_BF16) {
     auto k = absorb_query_kernel<__nv_bfloat16>;
-    if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (smem > 48 * 1024) ensure_max_smem(k, smem);
     return launch_pdl(k, grid, block, smem, st, sh.B, sh.H, sh.d_h, sh.d_n, sh.d_r, c,
                       (const __nv_bfloat16*)q, (const __nv_bfloat16*)M, q_pos, q_abs, rt,
                       early_trigger ? 1 : 0);
   }
   auto k = absorb_query_kernel<float>;
-  if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (smem > 48 * 1024) ensure_max_smem(k, smem);
   return launch_pdl(k, grid, block, smem, st, sh.B, sh.H, sh.d_h, sh.d_n, sh.d_r, c, (const float*)q,
                     (const float*)M, q_pos, q_abs, rt, early_trigger ? 1 : 0);
 }
@@ -302,7 +519,7 @@ static cudaError_t launch_prep_t(const gva_shape_t& sh, const void* q, const voi
   if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
   const size_t smem = sh.B > 0 ? absorb_smem_bytes(sh) : 0;
   auto k = prep_step_kernel<TQ, T>;
-  if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (smem > 48 * 1024) ensure_max_smem(k, smem);
   return launch_pdl(k, dim3((unsigned)blocks), dim3(256), smem, st, n_absorb, ay, az, sh.B, sh.H,
                     sh.d_h, sh.d_n, sh.d_r, c, (const TQ*)q, (const TQ*)M, q_pos, q_abs, N,
                     sh.G * sh.d_h, (const T*)v_new, (const T*)kpe_new, slot, pos, num_slots,

@@ -65,41 +65,53 @@ def lib() -> ctypes.CDLL:
     """Load libgva.so once; raise if it has not been built."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
-                               "`python -m compressed_kv_cache_gva_b200._build`")
-        L = ctypes.CDLL(LIB_PATH)
-        P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
-        SP = ctypes.POINTER(Shape)
-        L.gva_status_string.restype = ctypes.c_char_p
-        L.gva_status_string.argtypes = [ctypes.c_int]
-        L.gva_last_error.restype = ctypes.c_char_p
-        L.gva_last_error.argtypes = []
-        L.gva_absorb_query.restype = ctypes.c_int
-        L.gva_absorb_query.argtypes = [SP, P, P, P, P, P]
-        L.gva_append_cache.restype = ctypes.c_int
-        L.gva_append_cache.argtypes = [SP, I32, P, P, P, P, I64, P, P, P, P]
-        L.gva_decode_workspace_size.restype = SZ
-        L.gva_decode_workspace_size.argtypes = [SP, I64]
-        L.gva_decode_attention.restype = ctypes.c_int
-        L.gva_decode_attention.argtypes = [SP, P, P, P, P, P, I64, I64, P, P, P, SZ, P]
-        L.gqa_decode_attention.restype = ctypes.c_int
-        L.gqa_decode_attention.argtypes = [SP, P, P, P, P, P, I64, I64, P, P, P, SZ, P]
-        L.gva_decode_step.restype = ctypes.c_int
-        L.gva_decode_step.argtypes = [SP, P, P, P, I32, P, P, P, P, P, P, I64, P, P, I64, P, P, P, P,
-                                      P, SZ, P]
-        L.gva_decode_workspace_size_multi.restype = SZ
-        L.gva_decode_workspace_size_multi.argtypes = [SP, I32, I64]
-        L.gva_decode_attention_multi.restype = ctypes.c_int
-        L.gva_decode_attention_multi.argtypes = [SP, I32, P, P, P, P, P, I64, I64, P, P, P, SZ, P]
-        L.gva_merge_states.restype = ctypes.c_int
-        L.gva_merge_states.argtypes = [SP, I32, P, P, P, P, P]
-        L.gva_shared_kv_decode_attention.restype = ctypes.c_int
-        L.gva_shared_kv_decode_attention.argtypes = [SP, P, P, P, P, I64, I64, P, P, P, SZ, P]
-        L.gva_decode_attention_noalloc.restype = ctypes.c_int
-        L.gva_decode_attention_noalloc.argtypes = [SP, P, P, P, P, P, I64, I64, P, P, P]
-        _lib = L
+        _lib = load(LIB_PATH)
     return _lib
+
+
+def load(path: str) -> ctypes.CDLL:
+    """Open a build of the library and declare its C signatures."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m compressed_kv_cache_gva_b200._build`")
+    L = ctypes.CDLL(path)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    SP = ctypes.POINTER(Shape)
+    L.gva_status_string.restype = ctypes.c_char_p
+    L.gva_status_string.argtypes = [ctypes.c_int]
+    L.gva_last_error.restype = ctypes.c_char_p
+    L.gva_last_error.argtypes = []
+    L.gva_absorb_query.restype = ctypes.c_int
+    L.gva_absorb_query.argtypes = [SP, P, P, P, P, P]
+    L.gva_append_cache.restype = ctypes.c_int
+    L.gva_append_cache.argtypes = [SP, I32, P, P, P, P, I64, P, P, P, P]
+    L.gva_decode_workspace_size.restype = SZ
+    L.gva_decode_workspace_size.argtypes = [SP, I64]
+    L.gva_decode_attention.restype = ctypes.c_int
+    L.gva_decode_attention.argtypes = [SP, P, P, P, P, P, I64, I64, P, P, P, SZ, P]
+    L.gqa_decode_attention.restype = ctypes.c_int
+    L.gqa_decode_attention.argtypes = [SP, P, P, P, P, P, I64, I64, P, P, P, SZ, P]
+    L.gva_decode_step.restype = ctypes.c_int
+    L.gva_decode_step.argtypes = [SP, P, P, P, I32, P, P, P, P, P, P, I64, P, P, I64, P, P, P, P,
+                                  P, SZ, P]
+    L.gva_decode_workspace_size_multi.restype = SZ
+    L.gva_decode_workspace_size_multi.argtypes = [SP, I32, I64]
+    L.gva_decode_attention_multi.restype = ctypes.c_int
+    L.gva_decode_attention_multi.argtypes = [SP, I32, P, P, P, P, P, I64, I64, P, P, P, SZ, P]
+    L.gva_merge_states.restype = ctypes.c_int
+    L.gva_merge_states.argtypes = [SP, I32, P, P, P, P, P]
+    L.gva_shared_kv_decode_attention.restype = ctypes.c_int
+    L.gva_shared_kv_decode_attention.argtypes = [SP, P, P, P, P, I64, I64, P, P, P, SZ, P]
+    L.gqa_append_cache.restype = ctypes.c_int
+    L.gqa_append_cache.argtypes = [SP, I32, P, P, P, P, I64, P, P, P, P]
+    L.gqa_decode_step.restype = ctypes.c_int
+    L.gqa_decode_step.argtypes = [SP, P, P, I32, P, P, P, P, P, P, I64, P, P, I64, P, P, P, P,
+                                  P, SZ, P]
+    L.gva_decode_attention_noalloc.restype = ctypes.c_int
+    L.gva_decode_attention_noalloc.argtypes = [SP, P, P, P, P, P, I64, I64, P, P, P]
+    L.gva_noalloc_status.restype = ctypes.c_int
+    L.gva_noalloc_status.argtypes = [P, P]
+    return L
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -169,6 +181,25 @@ def gqa_decode_attention(shape: Shape, q, K_cache, V_cache, seq_offset, seq_len,
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def gqa_append_cache(shape: Shape, k_new, v_new, slot, pos, K_cache, V_cache, err_flag=None,
+                     stream=None):
+    """gqa_append_cache: the same-shape GQA baseline's append (key rotated over d_h)."""
+    _check(lib().gqa_append_cache(ctypes.byref(shape), slot.numel(), _ptr(k_new), _ptr(v_new),
+                                  _ptr(slot), _ptr(pos), V_cache.shape[0], _ptr(K_cache),
+                                  _ptr(V_cache), _ptr(err_flag), _stream(stream)))
+
+
+def gqa_decode_step(shape: Shape, q, q_pos, k_new, v_new, slot, pos, K_cache, V_cache,
+                    seq_offset, seq_len, max_total_tokens: int, q_rot, out, lse=None,
+                    err_flag=None, workspace=None, stream=None):
+    """gqa_decode_step: rotate the queries, append the new tokens, GQA decode."""
+    _check(lib().gqa_decode_step(
+        ctypes.byref(shape), _ptr(q), _ptr(q_pos), slot.numel(), _ptr(k_new), _ptr(v_new),
+        _ptr(slot), _ptr(pos), _ptr(K_cache), _ptr(V_cache), V_cache.shape[0], _ptr(seq_offset),
+        _ptr(seq_len), int(max_total_tokens), _ptr(q_rot), _ptr(out), _ptr(lse), _ptr(err_flag),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
 def decode_step(shape: Shape, q, M, q_pos, v_new, kpe_new, slot, pos, V_cache, kr_cache,
                 seq_offset, seq_len, max_total_tokens: int, q_abs, out, lse=None, err_flag=None,
                 workspace=None, stream=None):
@@ -225,8 +256,17 @@ def decode_attention_noalloc(shape: Shape, q_abs, V_cache, kr_cache, seq_offset,
         _stream(stream)))
 
 
+def noalloc_status(stream=None) -> int:
+    """Device status word of the last gva_decode_attention_noalloc call on the
+    current device (enqueued behind it on the stream; synchronises to read it)."""
+    buf = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _check(lib().gva_noalloc_status(_ptr(buf), _stream(stream)))
+    return int(buf.item())
+
+
 EXPORTS = ["gva_status_string", "gva_last_error", "gva_absorb_query", "gva_append_cache",
            "gva_decode_workspace_size", "gva_decode_attention", "gqa_decode_attention",
            "gva_decode_step", "gva_merge_states", "gva_decode_workspace_size_multi",
            "gva_decode_attention_multi", "gva_decode_attention_noalloc",
-           "gva_shared_kv_decode_attention"]
+           "gva_shared_kv_decode_attention", "gqa_append_cache", "gqa_decode_step",
+           "gva_noalloc_status"]

@@ -49,6 +49,31 @@ def shard_cache(V, k_rope, seq_offset, seq_len, world: int, rank: int, extra_slo
             torch.from_numpy(count.astype(np.int32)), start)
 
 
+def shard_step_inputs(V, k_rope, seq_offset, hist_len, append, world: int, rank: int):
+    """This rank's part of one decode step whose every sequence is split across
+    `world` ranks.  The step attends hist_len[b] + 1 rows (the history plus the
+    token appended in this step); rank r keeps positions
+    [(L+1)*r/world, (L+1)*(r+1)/world) of them, so exactly one rank holds the new
+    token's position L = hist_len[b] and appends it there.
+
+    V, k_rope, seq_offset: the full cache (host tensors), with a free slot after
+    each sequence's history; append = (v_new, kpe_new, slot, pos) of the B new
+    tokens.  Returns (V_r, k_rope_r, seq_offset_r, seq_len_r, append_r, start):
+    the compact shard, its step lengths, and the append inputs of the tokens that
+    land on this rank with their slots in the shard's layout."""
+    L = np.asarray(hist_len, dtype=np.int64)
+    step_len = torch.from_numpy((L + 1).astype(np.int32))
+    V_r, K_r, off_r, len_r, start = shard_cache(V, k_rope, seq_offset, step_len, world, rank)
+    cnt = len_r.numpy().astype(np.int64)
+    own = (L >= start) & (L < start + cnt)
+    sel = torch.from_numpy(own)
+    v_new, kpe_new, _, pos = append
+    slot_r = (off_r.numpy().astype(np.int64) + L - start)[own].astype(np.int32)
+    append_r = (v_new[sel].contiguous(), kpe_new[sel].contiguous(), torch.from_numpy(slot_r),
+                pos[sel].contiguous())
+    return V_r, K_r, off_r, len_r, append_r, start
+
+
 class SequenceSplitMerge:
     """Buffers and calls for the exchange + merge of one decode step.
 
@@ -67,9 +92,23 @@ class SequenceSplitMerge:
             self.out_part = torch.empty(B, H, d_h, dtype=torch.float32, device=device)
             self.lse_part = torch.empty(B, H, dtype=torch.float32, device=device)
 
+    def exchange(self):
+        """All-gather every rank's (out_part, lse_part) into outs/lses, in rank
+        order.  The buffers are gathered as flat vectors, which NCCL and gloo both
+        accept; with gloo, device buffers go through host copies."""
+        if self.world == 1:
+            return
+        import torch.distributed as dist
+        pairs = ((self.outs, self.out_part), (self.lses, self.lse_part))
+        if dist.get_backend(self.group) == "gloo" and self.outs.is_cuda:
+            for full, part in pairs:
+                host = torch.empty(full.numel(), dtype=full.dtype)
+                dist.all_gather_into_tensor(host, part.reshape(-1).cpu(), group=self.group)
+                full.copy_(host.view(full.shape))
+            return
+        for full, part in pairs:
+            dist.all_gather_into_tensor(full.view(-1), part.view(-1), group=self.group)
+
     def merge(self, out, lse=None):
-        if self.world > 1:
-            import torch.distributed as dist
-            dist.all_gather_into_tensor(self.outs, self.out_part, group=self.group)
-            dist.all_gather_into_tensor(self.lses, self.lse_part, group=self.group)
+        self.exchange()
         gva.merge_states(self.shape, self.outs, self.lses, out, lse)

@@ -193,6 +193,28 @@ def make_gqa_inputs(wl: Workload, extra_slots: int = 0,
                      num_slots=S)
 
 
+@dataclasses.dataclass
+class GQAAppendInputs:
+    k_new: torch.Tensor     # [N, G, d_h] raw (unrotated) key
+    v_new: torch.Tensor     # [N, G, d_h]
+    slot: torch.Tensor      # int32 [N]
+    pos: torch.Tensor       # int32 [N]
+
+
+def make_gqa_append_inputs(wl: Workload, slot: np.ndarray, pos: np.ndarray,
+                           seed: int = 3) -> GQAAppendInputs:
+    """New tokens for the same-shape GQA cache: key and value rows drawn as float32
+    standard normals (key first), rounded to the workload's storage type."""
+    rng = np.random.default_rng(seed)
+    N = len(slot)
+    f32 = np.float32
+    k = rng.standard_normal((N, wl.G, wl.d_h), dtype=f32)
+    v = rng.standard_normal((N, wl.G, wl.d_h), dtype=f32)
+    return GQAAppendInputs(k_new=_round(k, wl.dtype), v_new=_round(v, wl.dtype),
+                           slot=torch.from_numpy(np.asarray(slot, dtype=np.int32)),
+                           pos=torch.from_numpy(np.asarray(pos, dtype=np.int32)))
+
+
 def as_f64(t: torch.Tensor) -> np.ndarray:
     """Exact widening of a stored tensor to float64 for the oracle."""
     return t.detach().to("cpu").to(torch.float64).numpy()

@@ -184,6 +184,56 @@ gva_status_t gqa_decode_attention(const gva_shape_t* shape, const void* q, const
                                   size_t ws_bytes, void* stream);
 
 /*
+ * gqa_append_cache — persist N new tokens into the same-shape GQA cache, the
+ * matched baseline that keeps a key AND a value per group and token (onedev.kr
+ * review, "What differs": N_GQA = 2*T*G*d_h).  The value is copied bit-exactly;
+ * each group's key is rotated by the token's position over the whole head width
+ * (pair i with i + d_h/2, angle pos * rope_base^(-2i/d_h) in float64) and stored
+ * rounded once (to nearest, ties to even) to the cache type.
+ *
+ *   k_new, v_new      device [N, G, d_h] cache_dtype (k_new unrotated)
+ *   slot, pos         device [N] int32: destination slot and position of each token
+ *   K_cache, V_cache  device [num_slots, G, d_h] cache_dtype, updated in place
+ *   err_flag          device int32 or NULL: set to 1 if a slot lies outside
+ *                     [0, num_slots); such tokens are skipped, the others written
+ * Shape: d_n and d_r are ignored; d_h even and <= 128; rope_base > 0.
+ * Alignment: 16 bytes for every pointer; G*d_h*elt a multiple of 16 bytes.
+ * Errors: GVA_ERR_INVALID_ARG, GVA_ERR_UNSUPPORTED (odd or too wide d_h).
+ * N == 0 is a no-op.  Two tokens with the same slot race.
+ */
+gva_status_t gqa_append_cache(const gva_shape_t* shape, int32_t N, const void* k_new,
+                              const void* v_new, const int32_t* slot, const int32_t* pos,
+                              int64_t num_slots, void* K_cache, void* V_cache, int32_t* err_flag,
+                              void* stream);
+
+/*
+ * gqa_decode_step — one full decode step of the same-shape GQA baseline, the
+ * counterpart of gva_decode_step used to compare whole steps: the query of every
+ * sequence is rotated over d_h at q_pos[b] into q_rot (float32, unscaled), the
+ * n_new new tokens are appended as by gqa_append_cache, then gqa_decode_attention
+ * runs on q_rot (onedev.kr review, "What differs": GQA caches and reads a key and
+ * a value per group and token).  One kernel does the rotation and the append; the
+ * decode is launched behind it and streams every cache tile that holds no new
+ * slot before that kernel finishes.
+ *
+ *   q       device [B, H, d_h] q_dtype, unrotated;  q_pos device [B] int32
+ *   q_rot   device [B, H, d_h] float32, written (the rotated query)
+ *   k_new, v_new, slot, pos, K_cache, V_cache, num_slots, err_flag: as gqa_append_cache
+ *   seq_offset, seq_len, max_total_tokens, out, lse, workspace: as
+ *           gqa_decode_attention (seq_len already counts the new tokens; the
+ *           workspace size is gva_decode_workspace_size of the shape)
+ * Errors as gqa_append_cache and gqa_decode_attention; all validation happens
+ * before the first launch.
+ */
+gva_status_t gqa_decode_step(const gva_shape_t* shape, const void* q, const int32_t* q_pos,
+                             int32_t n_new, const void* k_new, const void* v_new,
+                             const int32_t* slot, const int32_t* pos, void* K_cache,
+                             void* V_cache, int64_t num_slots, const int32_t* seq_offset,
+                             const int32_t* seq_len, int64_t max_total_tokens, float* q_rot,
+                             void* out, float* lse, int32_t* err_flag, void* workspace,
+                             size_t ws_bytes, void* stream);
+
+/*
  * gva_decode_step — one full GVA decode step: gva_append_cache of the n_new new
  * tokens, gva_absorb_query, then gva_decode_attention, enqueued on `stream` in
  * that order (onedev.kr review, "How it works" and "What differs": the new
@@ -299,7 +349,10 @@ gva_status_t gva_merge_states(const gva_shape_t* shape, int32_t R, const float* 
  *   the scratch's device address cannot be found.
  *   The first call on each device looks up the scratch's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call before
- *   any stream capture.  Every call clears the scratch's status word on `stream`.
+ *   any stream capture.  Every accepted call zeroes the scratch's status word on
+ *   `stream` before its kernels run; a call rejected on the host enqueues nothing
+ *   and leaves the scratch untouched.  The call's device errors (GVA_DEVERR_*) stay
+ *   in that word until the next call: read them with gva_noalloc_status.
  *   All calls on a device share the one scratch array, which keeps the last call's
  *   contents: calls whose executions overlap on the GPU (different streams, or
  *   concurrent graphs) race and give wrong results.  Serialise them.
@@ -311,6 +364,25 @@ gva_status_t gva_decode_attention_noalloc(const gva_shape_t* shape, const float*
                                           const int32_t* seq_offset, const int32_t* seq_len,
                                           int64_t max_total_tokens, int64_t num_slots, void* out,
                                           float* lse, void* stream);
+
+/*
+ * gva_noalloc_status — the device status word of the most recent
+ * gva_decode_attention_noalloc call on the current device, i.e. the first 4 bytes
+ * of its static scratch: 0, or a GVA_DEVERR_* bit mask (GVA_DEVERR_RANGE: a
+ * sequence reached outside [0, num_slots) and its missing rows read as 0;
+ * GVA_DEVERR_WAIT: a bounded pipeline wait gave up and the outputs are invalid).
+ * The paper has no counterpart: an interface convenience of this library for
+ * callers without a workspace of their own.
+ *
+ *   status_out  device memory or page-locked host memory, one int32: receives
+ *               the word by an asynchronous copy enqueued on `stream`; it is valid
+ *               once the stream reaches that point (e.g. after
+ *               cudaStreamSynchronize).  Enqueue it behind the decode it checks,
+ *               on the same stream, and before the next no-allocation decode.
+ * Allocates nothing.  Errors: GVA_ERR_INVALID_ARG (NULL status_out), GVA_ERR_CUDA
+ * (the scratch's address or the copy failed).
+ */
+gva_status_t gva_noalloc_status(int32_t* status_out, void* stream);
 
 #ifdef __cplusplus
 }  /* extern "C" */

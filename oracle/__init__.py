@@ -5,7 +5,7 @@ this package.  The CUDA product path never does, and fails loudly without its
 compiled library instead of falling back here.
 """
 from .gva_oracle import (absorbed_query, append_cache, cache_scalars_gqa, cache_scalars_gva,
-                         gqa_decode, gva_decode, gva_decode_multi, rope, round_to_bf16, round_to_storage)
+                         gqa_append_cache, gqa_decode, gva_decode, gva_decode_multi, rope, round_to_bf16, round_to_storage)
 
 __all__ = ["absorbed_query", "append_cache", "cache_scalars_gqa", "cache_scalars_gva",
-           "gqa_decode", "gva_decode", "gva_decode_multi", "rope", "round_to_bf16", "round_to_storage"]
+           "gqa_append_cache", "gqa_decode", "gva_decode", "gva_decode_multi", "rope", "round_to_bf16", "round_to_storage"]

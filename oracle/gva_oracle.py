@@ -160,6 +160,30 @@ def append_cache(V_cache: np.ndarray, kr_cache: np.ndarray, v_new: np.ndarray,
     return V, KR, err
 
 
+def gqa_append_cache(K_cache: np.ndarray, V_cache: np.ndarray, k_new: np.ndarray,
+                     v_new: np.ndarray, slot: np.ndarray, pos: np.ndarray, base: float,
+                     dtype: str) -> Tuple[np.ndarray, np.ndarray, int]:
+    """Append for the matched GQA baseline, which caches a key and a value per
+    group and token (onedev.kr review, "What differs": N_GQA = 2*T*G*d_h).  Plain
+    RoPE acts on the whole key, so every group's key of width d_h is rotated by
+    the token's position (the same rotation as ``rope``, over d_h) and stored in
+    the cache type; the value is stored unchanged.  Slots outside [0, S) are
+    skipped and reported through the returned flag.  Returns new copies of K and V."""
+    K = np.array(K_cache, dtype=np.float64, copy=True)
+    V = np.array(V_cache, dtype=np.float64, copy=True)
+    S = K.shape[0]
+    err = 0
+    for i in range(len(slot)):
+        s = int(slot[i])
+        if s < 0 or s >= S:
+            err = 1
+            continue
+        V[s] = np.asarray(v_new[i], dtype=np.float64)
+        K[s] = round_to_storage(rope(np.asarray(k_new[i], dtype=np.float64), float(pos[i]), base),
+                                dtype)
+    return K, V, err
+
+
 # ----------------------------------------------------------------------------
 # Decode attention, non-absorbed route
 # ----------------------------------------------------------------------------

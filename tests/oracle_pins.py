@@ -255,6 +255,42 @@ def check_append(orc):
     assert np.max(np.abs(K1[2] - orc.rope(k[0], 5.0, 10000.0))) < 1e-6         # float32 storage
 
 
+def check_gqa_append(orc):
+    """The GQA baseline's append: each group's key equals transformers' Llama rotary
+    embedding over the full head width at the token's position (an implementation
+    independent of the oracle's), rounded once to bf16; the value is copied; slots
+    outside the cache are skipped and flagged."""
+    from transformers import LlamaConfig
+    from transformers.models.llama.modeling_llama import LlamaRotaryEmbedding, apply_rotary_pos_emb
+    rng = np.random.default_rng(22)
+    for d_h, G, base in ((8, 2, 10000.0), (64, 4, 10000.0), (128, 2, 500000.0)):
+        S = 9
+        K0 = orc.round_to_bf16(rng.standard_normal((S, G, d_h)))
+        V0 = orc.round_to_bf16(rng.standard_normal((S, G, d_h)))
+        k = orc.round_to_bf16(rng.standard_normal((4, G, d_h)))
+        v = orc.round_to_bf16(rng.standard_normal((4, G, d_h)))
+        slot, pos = np.array([3, 8, -1, 0]), np.array([0, 4093, 5, 77])
+        K1, V1, err = orc.gqa_append_cache(K0, V0, k, v, slot, pos, base, "bf16")
+        assert err == 1
+        cfg = LlamaConfig(hidden_size=4 * d_h, num_attention_heads=4, head_dim=d_h, rope_theta=base)
+        emb = LlamaRotaryEmbedding(cfg)
+        for i in (0, 1, 3):
+            xt = torch.from_numpy(k[i])[None, :, None, :]            # [1, G, 1, d_h]
+            cos, sin = emb(xt, torch.tensor([[int(pos[i])]]))
+            ref, _ = apply_rotary_pos_emb(xt, xt, cos, sin)
+            ref = ref[0, :, 0].numpy()
+            s_ = slot[i]
+            # transformers forms its angles in float32: compare before the bf16
+            # rounding can amplify that, then check the stored value is a bf16
+            assert np.max(np.abs(K1[s_] - ref)) <= 4e-3 * max(1.0, np.max(np.abs(ref))), (d_h, i)
+            assert np.array_equal(orc.round_to_bf16(K1[s_]), K1[s_])
+            assert np.array_equal(V1[s_], v[i])
+        assert np.array_equal(K1[3], k[0])                           # position 0: unrotated
+        untouched = [j for j in range(S) if j not in (3, 8, 0)]
+        assert np.array_equal(K1[untouched], K0[untouched])
+        assert np.array_equal(V1[untouched], V0[untouched])
+
+
 def check_multi_query_causal(orc):
     """Several new tokens decoded together: one query reduces to the one-token
     decode; the last query sees the whole cache; query i does not see rows after
@@ -283,4 +319,4 @@ def check_multi_query_causal(orc):
 ALL_CHECKS = [check_cache_ratio, check_kv_shared_is_sdpa, check_gqa_is_sdpa, check_rope_matches_llama,
               check_relative_position, check_rope_group_law, check_absorption_identity,
               check_softmax_closed_forms, check_bruteforce, check_round_to_bf16, check_append,
-              check_multi_query_causal]
+              check_multi_query_causal, check_gqa_append]

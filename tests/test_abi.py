@@ -131,6 +131,31 @@ def test_shared_kv_needs_keys_equal_to_values(L):
         assert st == 1 and b"shared keys and values" in L.gva_last_error()
 
 
+def test_gqa_append_and_step_validate_on_the_host(L):
+    """The GQA baseline's append and step reject, before any launch, a head width
+    its RoPE cannot rotate (odd or above 128), a non-positive RoPE base, NULL
+    pointers and misaligned ones; N = 0 appends nothing."""
+    for bad, code in ((dict(d_h=130, d_n=130, d_r=0), 2), (dict(d_h=72, d_n=72, d_r=0, G=2, H=8), 0),
+                      (dict(d_h=64, d_n=64, d_r=0, rope_base=-1.0), 1)):
+        sh = _shape(**bad)
+        st = L.gqa_append_cache(ctypes.byref(sh), 4, FAKE, FAKE, FAKE, FAKE, 10, FAKE, FAKE, None,
+                                None)
+        if code == 0:      # a valid shape: only the fake pointers stop it (no device here)
+            continue
+        assert st == code, (bad, st)
+    sh = _shape(d_h=64, d_n=64, d_r=0)
+    st = L.gqa_append_cache(ctypes.byref(sh), 4, None, FAKE, FAKE, FAKE, 10, FAKE, FAKE, None, None)
+    assert st == 1 and b"NULL" in L.gva_last_error()
+    st = L.gqa_append_cache(ctypes.byref(sh), 4, FAKE + 2, FAKE, FAKE, FAKE, 10, FAKE, FAKE, None,
+                            None)
+    assert st == 1 and b"aligned" in L.gva_last_error()
+    assert L.gqa_append_cache(ctypes.byref(sh), 0, None, None, None, None, 1, None, None, None,
+                              None) == 0
+    st = L.gqa_decode_step(ctypes.byref(sh), FAKE, FAKE, 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 10,
+                           FAKE, FAKE, 100, None, FAKE, None, None, FAKE, 1 << 20, None)
+    assert st == 1 and b"NULL" in L.gva_last_error()
+
+
 def test_missing_library_fails_loudly(tmp_path):
     """No fallback: without the compiled library the binding raises on first use."""
     import subprocess

@@ -83,57 +83,76 @@ def _split_worker(rank, world, port, q):
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
     try:
-        import oracle
-        from compressed_kv_cache_gva_b200 import seqsplit
-        from compressed_kv_cache_gva_b200.synth import WORKLOADS, as_f64, make_decode_inputs
+        from compressed_kv_cache_gva_b200 import gva, seqsplit
+        from compressed_kv_cache_gva_b200.synth import (WORKLOADS, make_append_inputs,
+                                                        make_decode_inputs)
         wl = WORKLOADS["350m_b8_t4096"]
-        L = np.array([5, 64, 1, 33])
-        di = make_decode_inputs(wl, lengths=L)
-        V_r, K_r, off_r, len_r, start = seqsplit.shard_cache(di.V, di.k_rope, di.seq_offset,
-                                                             di.seq_len, world, rank)
-        out_r, lse_r = oracle.gva_decode(as_f64(di.q), as_f64(di.M), di.q_pos.numpy(), as_f64(V_r),
-                                         as_f64(K_r), off_r.numpy(), len_r.numpy(), wl.d_n,
-                                         wl.d_r, wl.rope_base)
-        outs = [torch.zeros(out_r.shape, dtype=torch.float64) for _ in range(world)]
-        lses = [torch.zeros(lse_r.shape, dtype=torch.float64) for _ in range(world)]
-        dist.all_gather(outs, torch.from_numpy(out_r))
-        dist.all_gather(lses, torch.from_numpy(lse_r))
-        if rank == 0:
-            q.put((np.stack([o.numpy() for o in outs]), np.stack([l.numpy() for l in lses])))
+        L = np.array([5, 64, 1, 33, 0])
+        di = make_decode_inputs(wl, extra_slots=1, lengths=L)
+        slots = (di.seq_offset.numpy() + L).astype(np.int32)
+        ap = make_append_inputs(wl, slots, L.astype(np.int32))
+        V_r, K_r, off_r, len_r, app_r, start = seqsplit.shard_step_inputs(
+            di.V, di.k_rope, di.seq_offset, L, (ap.v_new, ap.kpe_new, ap.slot, ap.pos), world, rank)
+        # the product's exchange on host buffers: each rank's part is a recognisable
+        # function of its rank, gathered into every rank's outs / lses in rank order
+        sh = gva.make_shape(len(L), wl.H, wl.G, wl.d_h, wl.d_n, wl.d_r)
+        m = seqsplit.SequenceSplitMerge(sh, world, "cpu")
+        m.out_part.copy_(torch.arange(m.out_part.numel(), dtype=torch.float32).view_as(m.out_part)
+                         + 1000 * rank)
+        m.lse_part.fill_(-float(rank))
+        m.exchange()
+        q.put((rank, start, len_r.numpy(), off_r.numpy(), V_r.float().numpy(), K_r.float().numpy(),
+               [t.float().numpy() if t.is_floating_point() else t.numpy() for t in app_r],
+               m.outs.numpy(), m.lses.numpy()))
     finally:
         dist.destroy_process_group()
 
 
-def test_sequence_split_exchange_world_size_2():
-    """Each rank decodes its part of every sequence (oracle on CPU), the parts
-    are all-gathered in rank order and merged by the softmax decomposition; the
-    result equals the oracle on the whole cache."""
+def test_sequence_split_shards_and_exchange_world_size_2():
+    """The sequence split's host logic on two gloo ranks: shard_step_inputs cuts
+    every sequence's step (history + the appended token) into two parts that
+    partition its positions, only the rank holding position L appends the new
+    token (at the right slot of its shard), and SequenceSplitMerge.exchange gives
+    every rank all parts in rank order.  (The merge arithmetic and the per-rank
+    decodes run on the GPU: tests/test_gpu_seqsplit_ranks.py.)"""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
     procs = [ctx.Process(target=_split_worker, args=(r, 2, port, q)) for r in range(2)]
     for p in procs:
         p.start()
-    outs, lses = q.get(timeout=180)
+    res = sorted([q.get(timeout=180) for _ in range(2)], key=lambda x: x[0])
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
     sys.path.insert(0, ROOT)
-    import oracle
-    from compressed_kv_cache_gva_b200 import seqsplit
-    from compressed_kv_cache_gva_b200.synth import WORKLOADS, as_f64, make_decode_inputs
+    from compressed_kv_cache_gva_b200.synth import (WORKLOADS, make_append_inputs,
+                                                    make_decode_inputs)
     wl = WORKLOADS["350m_b8_t4096"]
-    L = np.array([5, 64, 1, 33])
-    di = make_decode_inputs(wl, lengths=L)
-    ref, ref_lse = oracle.gva_decode(as_f64(di.q), as_f64(di.M), di.q_pos.numpy(), as_f64(di.V),
-                                     as_f64(di.k_rope), di.seq_offset.numpy(), L, wl.d_n, wl.d_r,
-                                     wl.rope_base)
-    # the parts partition the positions
-    s0, c0 = seqsplit.shard_ranges(L, 2, 0)
-    s1, c1 = seqsplit.shard_ranges(L, 2, 1)
-    assert np.array_equal(s0, 0 * L) and np.array_equal(s1, c0) and np.array_equal(c0 + c1, L)
-    mx = np.max(lses, axis=0)
-    w = np.where(np.isneginf(lses), 0.0, np.exp(lses - mx))
-    merged = (w[..., None] * np.nan_to_num(outs)).sum(0) / w.sum(0)[..., None]
-    assert np.max(np.abs(merged - ref)) < 1e-12
-    assert np.max(np.abs(mx + np.log(w.sum(0)) - ref_lse)) < 1e-12
+    L = np.array([5, 64, 1, 33, 0])
+    di = make_decode_inputs(wl, extra_slots=1, lengths=L)
+    ap = make_append_inputs(wl, (di.seq_offset.numpy() + L).astype(np.int32), L.astype(np.int32))
+    V = di.V.float().numpy()
+    KR = di.k_rope.float().numpy()
+    off = di.seq_offset.numpy()
+    owners = np.zeros(len(L), dtype=int)
+    for rank, start, cnt, off_r, V_r, K_r, (v_new, kpe_new, slot_r, pos_r), outs, lses in res:
+        # parts of the step's L + 1 positions: rank 0 from 0, rank 1 from rank 0's end
+        assert np.array_equal(start, ((L + 1) * rank) // 2)
+        for b in range(len(L)):
+            rows = np.arange(off[b] + start[b], off[b] + start[b] + cnt[b])
+            assert np.array_equal(V_r[off_r[b]:off_r[b] + cnt[b]], V[rows])
+            assert np.array_equal(K_r[off_r[b]:off_r[b] + cnt[b]], KR[rows])
+        own = (L >= start) & (L < start + cnt)
+        owners += own
+        assert np.array_equal(slot_r, (off_r + L - start)[own])
+        assert np.array_equal(pos_r, L[own])
+        assert np.array_equal(v_new, ap.v_new.float().numpy()[own])
+        assert np.array_equal(kpe_new, ap.kpe_new.float().numpy()[own])
+        # every rank holds every part, in rank order
+        part = np.arange(outs[0].size, dtype=np.float32).reshape(outs[0].shape)
+        assert np.array_equal(outs[0], part) and np.array_equal(outs[1], part + 1000)
+        assert np.all(lses[0] == 0) and np.all(lses[1] == -1)
+    assert np.all(owners == 1)               # each new token is appended exactly once
+    total = sum(r[2] for r in res)
+    assert np.array_equal(total, L + 1)

@@ -146,6 +146,14 @@ def _mut_append_no_rotate(m):
     m.append_cache = bad
 
 
+def _mut_gqa_append_no_rotate(m):
+    orig = m.gqa_append_cache
+
+    def bad(K_cache, V_cache, k_new, v_new, slot, pos, base, dtype):   # key stored unrotated
+        return orig(K_cache, V_cache, k_new, v_new, slot, np.zeros_like(np.asarray(pos)), base, dtype)
+    m.gqa_append_cache = bad
+
+
 def _mut_causal_off_by_one(m):
     orig = m.gva_decode
 
@@ -166,7 +174,7 @@ def _mut_causal_off_by_one(m):
 MUTATIONS = [_mut_rope_sign, _mut_rope_adjacent_pairs, _mut_rope_freq, _mut_drop_rope_term,
              _mut_group_map, _mut_transposed_map, _mut_scale, _mut_softmax_no_norm,
              _mut_off_by_one_len, _mut_gqa_group_map, _mut_bf16_truncate, _mut_cache_count,
-             _mut_append_no_rotate, _mut_causal_off_by_one]
+             _mut_append_no_rotate, _mut_causal_off_by_one, _mut_gqa_append_no_rotate]
 
 
 @pytest.mark.parametrize("mutate", MUTATIONS, ids=lambda f: f.__name__[5:])
