@@ -122,6 +122,7 @@ struct Plan {
   bool mma;   // tensor-core split kernel (mma.sync or tcgen05)
   bool tc;    // the tcgen05 one
   int grid;
+  int pool;   // tail-pool tiles per CTA of the split kernel (0: none)
   gva::WsLayout ws;
 };
 
@@ -137,7 +138,8 @@ gva_status_t plan_decode(const gva_shape_t& sh, bool gqa, long long max_total, P
           gva::tc_decode_supported(sh);
   p->grid = p->tc ? gva::tc_decode_grid(sh, sms, max_total)
           : p->mma ? gva::mma_grid(sh, sms, max_total, gqa) : gva::simt_grid(sh, sms, max_total, gqa);
-  p->ws = gva::ws_layout(sh.B, sh.H, sh.d_h, p->grid);
+  p->pool = (p->mma && !p->tc) ? gva::kPoolTilesPerCta : 0;   // the mma.sync split kernel only
+  p->ws = gva::ws_layout(sh.B, sh.H, sh.d_h, p->grid, p->pool);
   return GVA_OK;
 }
 
@@ -176,7 +178,7 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
     return s;
   if (nq > 1 && !p.mma)
     return fail(GVA_ERR_UNSUPPORTED, "several query tokens need the tensor-core kernel "
-                "(bf16 cache, (H/G)*n_query in {4, 8}, d_h in {64, 128})");
+                "(bf16 cache, (H/G)*n_query <= 8, d_h in {64, 128})");
   if (ws_bytes < p.ws.total)
     return fail(GVA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, p.ws.total);
 
@@ -199,7 +201,9 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
   a.num_slots = num_slots;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.status = reinterpret_cast<int*>(ws);
-  a.meta = reinterpret_cast<int2*>(ws + p.ws.meta_off);
+  a.pool_ctr = reinterpret_cast<int*>(ws) + 1;
+  a.pool_per_cta = p.pool;
+  a.meta = reinterpret_cast<int4*>(ws + p.ws.meta_off);
   a.part_ml = reinterpret_cast<float2*>(ws + p.ws.ml_off);
   a.part_o = reinterpret_cast<float*>(ws + p.ws.o_off);
   a.grid = p.grid;
@@ -210,10 +214,11 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
   a.trace = g_trace;
 #endif
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // clear_status: zero the workspace's status word on the stream right before the
-  // split kernel, once every check has passed (a rejected call enqueues nothing)
+  // clear_status: zero the workspace's status word and pool counter on the stream
+  // right before the split kernel, once every check has passed (a rejected call
+  // enqueues nothing)
   auto clear = [&]() -> cudaError_t {
-    return clear_status ? cudaMemsetAsync(a.status, 0, sizeof(int), st) : cudaSuccess;
+    return clear_status ? cudaMemsetAsync(a.status, 0, 2 * sizeof(int), st) : cudaSuccess;
   };
 
   cudaError_t err;

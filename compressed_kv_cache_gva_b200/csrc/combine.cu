@@ -25,10 +25,15 @@ template <typename TO>
 __global__ void __launch_bounds__(1024)
     combine_kernel(const DecodeArgs a, TO* __restrict__ out, float* __restrict__ lse) {
   __shared__ float sm_m[32][33], sm_l[32][33], sm_o[32][33];
-  __shared__ int s_meta[2];
+  __shared__ int4 s_meta;
   const int b = blockIdx.x, h = blockIdx.y, d = blockIdx.z * 32 + (threadIdx.x & 31);
   const int H = a.H, d_h = a.d_h;
   const int tid = threadIdx.x, lane = tid & 31, pg = tid >> 5, npg = blockDim.x >> 5;
+  // The next kernel may launch at once: every kernel of this library waits for its
+  // predecessor before it reads what that one writes, so in a decode-step loop the
+  // next step's first kernel and split kernel start (and the split kernel streams
+  // its cache into SMs the finished split CTAs leave) while this combine runs.
+  pdl_trigger();
   const bool scan = a.B <= kCombineScanMaxB;
   if (scan && pg == 0) {
     // tokens of the whole batch, tiles of sequences < b, of b and of the batch
@@ -51,19 +56,18 @@ __global__ void __launch_bounds__(1024)
       nb += __shfl_xor_sync(0xffffffffu, nb, o);
     }
     if (lane == 0) {
-      int first = 0, count = 0;
+      int4 m = make_int4(0, 0, 0, 0);
       if (nb > 0 && total < (1ll << 31)) {
-        const TileSplit ts{(int)tiles, a.grid};
-        const int f = ts.cta_of((int)before), l = ts.cta_of((int)before + nb - 1);
-        first = f + b;
-        count = l - f + 1;
+        const TileSplit ts = make_split((int)tiles, a.grid, a.pool_per_cta);
+        m = ts.slots(b, (int)before, (int)before + nb, a.B);
       }
-      s_meta[0] = first;
-      s_meta[1] = count;
+      s_meta = m;
     }
   }
   pdl_wait();
-  pdl_trigger();
+  // the split kernel has completed: reset its pool counter for the next call
+  if (a.pool_ctr && tid == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+    *a.pool_ctr = 0;
 #ifdef GVA_TRACE
   const int cid = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
   if (a.trace && tid == 0 && cid < 16384) {
@@ -72,19 +76,20 @@ __global__ void __launch_bounds__(1024)
     a.trace[4096 * 8 + cid * 2] = tt;
   }
 #endif
-  int base, n;
+  int4 meta;
   if (scan) {
     __syncthreads();
-    base = s_meta[0];
-    n = s_meta[1];
+    meta = s_meta;
   } else {
-    const int2 meta = a.meta[b];
-    base = meta.x;
-    n = meta.y;
+    meta = a.meta[b];
   }
+  // pieces 0 .. sc-1 are the static slots meta.x + c, pieces sc .. n-1 the pool
+  // slots meta.z + c - sc, merged in this fixed order
+  const int sc = meta.y, n = meta.y + meta.w;
+  const int pool_shift = meta.z - meta.x - sc;
   const bool col = d < d_h;
-  const float2* ml = a.part_ml + (size_t)base * H + h;
-  const float* po = a.part_o + ((size_t)base * H + h) * d_h + (col ? d : 0);
+  const float2* ml = a.part_ml + (size_t)meta.x * H + h;
+  const float* po = a.part_o + ((size_t)meta.x * H + h) * d_h + (col ? d : 0);
   const size_t mstride = H, ostride = (size_t)H * d_h;
   float m = -INFINITY, l = 0.f, o = 0.f;
   for (int c0 = pg; c0 < n; c0 += kCombinePieces * npg) {
@@ -94,8 +99,9 @@ __global__ void __launch_bounds__(1024)
     for (int u = 0; u < kCombinePieces; ++u) {
       const int c = c0 + u * npg;
       if (c < n) {
-        e[u] = ml[(size_t)c * mstride];
-        x[u] = po[(size_t)c * ostride];
+        const long long sl = c < sc ? c : (long long)c + pool_shift;   // relative to meta.x
+        e[u] = ml[sl * (long long)mstride];
+        x[u] = po[sl * (long long)ostride];
       }
     }
 #pragma unroll
@@ -145,7 +151,7 @@ cudaError_t launch_combine(const gva_shape_t& sh, const DecodeArgs& a, void* out
   const dim3 grid(sh.B, sh.H, (sh.d_h + 31) / 32);
   // a sequence has about grid/B + 1 pieces (ragged batches: more for the long
   // ones); aim at ~kCombinePieces pieces per thread, 1..32 piece groups
-  const int per_seq = a.grid / (sh.B > 0 ? sh.B : 1) + 2;
+  const int per_seq = a.grid * (1 + a.pool_per_cta) / (sh.B > 0 ? sh.B : 1) + 2;
   int npg = (per_seq + kCombinePieces - 1) / kCombinePieces;
   npg = npg < 1 ? 1 : (npg > 32 ? 32 : npg);
   if (sh.out_dtype == GVA_BF16)
@@ -164,8 +170,8 @@ __global__ void __launch_bounds__(128)
                         const float* __restrict__ lses, TO* __restrict__ out,
                         float* __restrict__ lse) {
   const int bh = blockIdx.x;
+  pdl_trigger();   // as in the combine: successors wait before they read
   pdl_wait();
-  pdl_trigger();
   float mx = -INFINITY;
   for (int r = 0; r < R; ++r) mx = fmaxf(mx, lses[(size_t)r * BH + bh]);
   float z = 0.f;

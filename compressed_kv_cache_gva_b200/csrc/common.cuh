@@ -32,9 +32,28 @@ constexpr uint32_t kWaitLimit = GVA_WAIT_LIMIT;
 constexpr unsigned long long kWaitNs = GVA_WAIT_NS;
 
 // ---------------------------------------------------------------------------
-// Workspace: [status word | meta[B] | partial (m,l)[P][H] | partial o[P][H][d_h]]
-// P = grid + B partial slots: the piece of sequence b handled by CTA i lands in
-// slot i + b (unique, see worklist below).
+// Tail pool of the split (see TileSplit): when a batch has at least
+// kPoolMinTilesPerCta tiles per CTA, its last kPoolTilesPerCta * grid tiles are
+// not assigned statically; CTAs that finish their static range take them one at
+// a time.  0 disables the pool.
+// ---------------------------------------------------------------------------
+#ifndef GVA_POOL_TILES_PER_CTA
+#define GVA_POOL_TILES_PER_CTA 1
+#endif
+constexpr int kPoolTilesPerCta = GVA_POOL_TILES_PER_CTA;
+constexpr int kPoolMinTilesPerCta = 4;
+
+__host__ __device__ inline int pool_tiles(int NT, int grid, int per_cta) {
+  if (per_cta <= 0 || (long long)NT < (long long)kPoolMinTilesPerCta * grid) return 0;
+  const long long n = (long long)per_cta * grid;
+  return n < NT ? (int)n : NT;
+}
+
+// ---------------------------------------------------------------------------
+// Workspace: [status word, pool counter | meta[B] | partial (m,l)[P][H] |
+// partial o[P][H][d_h]].  P = grid * (1 + pool tiles per CTA) + B partial slots:
+// the static piece of sequence b handled by CTA i lands in slot i + b (unique,
+// see the work list below), pool tile v in slot grid + B + (v - NS).
 // ---------------------------------------------------------------------------
 struct WsLayout {
   size_t meta_off, ml_off, o_off, total;
@@ -42,11 +61,11 @@ struct WsLayout {
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline WsLayout ws_layout(int B, int H, int d_h, int grid) {
+__host__ __device__ inline WsLayout ws_layout(int B, int H, int d_h, int grid, int pool_per_cta) {
   WsLayout w;
-  size_t parts = (size_t)grid + (size_t)B;
+  size_t parts = (size_t)grid * (size_t)(1 + (pool_per_cta > 0 ? pool_per_cta : 0)) + (size_t)B;
   w.meta_off = 256;
-  w.ml_off = align_up(w.meta_off + sizeof(int2) * (size_t)B, 256);
+  w.ml_off = align_up(w.meta_off + sizeof(int4) * (size_t)B, 256);
   w.o_off = align_up(w.ml_off + sizeof(float2) * parts * (size_t)H, 256);
   w.total = align_up(w.o_off + sizeof(float) * parts * (size_t)H * (size_t)d_h, 256);
   return w;
@@ -65,7 +84,9 @@ struct DecodeArgs {
   const int* seq_len;
   long long num_slots;
   int* status;
-  int2* meta;                // per sequence: (first partial slot, number of pieces)
+  int* pool_ctr;             // tickets of the tail pool taken so far (the combine resets it)
+  int pool_per_cta;          // pool tiles per CTA of the split kernel (0: no pool)
+  int4* meta;                // per sequence: static slots (first, count), pool slots (first, count)
   float2* part_ml;           // [P][H] (running max, running sum), base-2
   float* part_o;             // [P][H][d_h] un-normalised output
   int nq;                    // query tokens per sequence (causal among them), >= 1
@@ -124,26 +145,57 @@ __device__ __forceinline__ void trace_tile(const DecodeArgs& a, int k, int which
 // (one tile each): cut over all of them, some CTAs would own no tile although they
 // sit inside a sequence's run of slots, and the combine would read slots that no
 // CTA wrote.  With NT >= grid, used() == grid and nothing changes.
+//
+// Tail pool: only the first NS tiles are cut this way; tiles [NS, NT) (the last
+// pool_tiles(...) of the batch) go to whichever CTA asks first once its static
+// range is issued, one tile per ticket from a counter in the workspace.  A CTA's
+// static range ends when its DRAM requests have been served, which varies by a
+// few tiles between CTAs; the pool lets the early ones absorb that spread.
+// Each pool tile keeps its own partial slot, so the merge order, and the result,
+// do not depend on which CTA took it.
 // ---------------------------------------------------------------------------
 struct TileSplit {
   int NT;     // tiles in the batch
   int grid;   // CTAs launched
-  // CTAs that own tiles; the rest own none
-  __device__ __forceinline__ int used() const { return grid < NT ? grid : (NT > 0 ? NT : 1); }
-  __device__ __forceinline__ bool narrow() const { return NT <= 0x7fffffff / used(); }
+  int NS;     // statically assigned tiles; [NS, NT) is the pool
+  // CTAs that own static tiles; the rest own none
+  __device__ __forceinline__ int used() const { return grid < NS ? grid : (NS > 0 ? NS : 1); }
+  __device__ __forceinline__ bool narrow() const { return NS <= 0x7fffffff / used(); }
   __device__ __forceinline__ int first(int i) const {
     const int g = used();
     i = i < g ? i : g;
-    return narrow() ? (int)((unsigned)(i * NT) / (unsigned)g)
-                    : (int)((long long)i * NT / g);
+    return narrow() ? (int)((unsigned)(i * NS) / (unsigned)g)
+                    : (int)((long long)i * NS / g);
   }
-  // the CTA that owns tile u (0 <= u < NT): the last i with first(i) <= u
+  // the CTA that owns static tile u (0 <= u < NS): the last i with first(i) <= u
   __device__ __forceinline__ int cta_of(int u) const {
     const int g = used();
-    return narrow() ? (int)((unsigned)((u + 1) * g - 1) / (unsigned)NT)
-                    : (int)(((long long)(u + 1) * g - 1) / NT);
+    return narrow() ? (int)((unsigned)((u + 1) * g - 1) / (unsigned)NS)
+                    : (int)(((long long)(u + 1) * g - 1) / NS);
+  }
+  __device__ __forceinline__ int pool() const { return NT - NS; }
+  // Partial slots of sequence b whose tiles are [t0, t1) in batch order:
+  // (first static slot, static count, first pool slot, pool count).
+  __device__ __forceinline__ int4 slots(int b, int t0, int t1, int B) const {
+    int4 m = make_int4(0, 0, 0, 0);
+    const int s1 = t1 < NS ? t1 : NS;
+    if (t0 < s1) {
+      const int f = cta_of(t0), l = cta_of(s1 - 1);
+      m.x = f + b;
+      m.y = l - f + 1;
+    }
+    const int u0 = t0 > NS ? t0 : NS;
+    if (u0 < t1) {
+      m.z = grid + B + (u0 - NS);
+      m.w = t1 - u0;
+    }
+    return m;
   }
 };
+
+__device__ __forceinline__ TileSplit make_split(int NT, int grid, int pool_per_cta) {
+  return TileSplit{NT, grid, NT - pool_tiles(NT, grid, pool_per_cta)};
+}
 
 // Exclusive prefix sums of val(0..B-1) (each >= 0) into prefix[0..B], for the
 // whole block; returns the total.  If the total does not fit in int, every
@@ -304,10 +356,9 @@ __device__ inline void write_meta(const DecodeArgs& a, const int* prefix, const 
                                   TileSplit ts) {
   for (int b = threadIdx.x; b < a.B; b += blockDim.x) {
     int L = prefix[b + 1] - prefix[b];
-    int2 m = make_int2(0, 0);
+    int4 m = make_int4(0, 0, 0, 0);
     if (L > 0) {
-      const int first = ts.cta_of(tp[b]), last = ts.cta_of(tp[b + 1] - 1);
-      m = make_int2(first + b, last - first + 1);
+      m = ts.slots(b, tp[b], tp[b + 1], a.B);
       long long off = __ldg(a.seq_offset + b);
       if (off < 0 || off + L > a.num_slots) atomicOr(a.status, GVA_DEVERR_RANGE);
     }
@@ -318,10 +369,15 @@ __device__ inline void write_meta(const DecodeArgs& a, const int* prefix, const 
 // ---------------------------------------------------------------------------
 // Programmatic dependent launch.  Every kernel here runs a prologue that reads
 // nothing the preceding kernel of the stream writes, then waits for that kernel
-// (griddepcontrol.wait: it has completed and its writes are visible), then lets
-// the next kernel start launching.  Since every kernel waits before it triggers,
-// a kernel can only start once the kernel two places earlier has completed, so
-// the chain stays ordered transitively.
+// (griddepcontrol.wait: it has completed and its writes are visible) before it
+// reads or writes anything a predecessor touches.  A kernel whose wait returned
+// knows its predecessor completed, and that one waited on its own predecessor,
+// so the chain stays ordered transitively.  The split kernels trigger their
+// successor after their wait; the first kernel of a fused step and the combine
+// trigger at entry, so the next split kernel can launch early: before its own
+// wait it only reads caller inputs and cache rows no kernel in flight writes.
+// A dependent launches only once every CTA of its predecessor has triggered, so
+// a waiting successor never holds the SM resources its predecessors still need.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {

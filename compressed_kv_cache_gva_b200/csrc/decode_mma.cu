@@ -20,7 +20,9 @@ cudaError_t run(const gva_shape_t& sh, DecodeArgs& a, const CUtensorMap& tx, con
 // default-constructed config type.  Returns false when none matches.
 template <class F>
 bool dispatch(const gva_shape_t& sh, bool gqa, F&& f) {
-  const int hpg = sh.H / sh.G;
+  // columns per group (heads per group x query tokens), padded up to 4 or 8
+  const int cols = sh.H / sh.G;
+  const int hpg = cols <= 4 ? 4 : (cols <= 8 ? 8 : -1);
   const int drp = gqa ? 0 : (sh.d_r == 0 ? 0 : (sh.d_r <= 16 ? 16 : (sh.d_r <= 32 ? 32 : -1)));
 #define GVA_CASE(DH, NG, HPG, DRP, GQ)                                                     \
   if (sh.d_h == DH && sh.G == NG && hpg == HPG && drp == DRP && gqa == GQ) {              \

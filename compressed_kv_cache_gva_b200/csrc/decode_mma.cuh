@@ -18,6 +18,9 @@
 //
 // For GQA (same-shape comparison) the scores operand is the K tile, a separate V
 // tile is streamed next to it and there is no positional key.
+// Groups with fewer query columns than 4 (H/G = 1, 2, 3 with one query token) run
+// the 4-column configuration and groups with 5..7 the 8-column one: the spare
+// columns carry a zero query, and their outputs are never stored.
 #pragma once
 
 #include "common.cuh"
@@ -135,10 +138,15 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
   if (scan_batch<C::TT>(a.seq_len, a.B, len_lane, prefix, tp, wtmp) >= (1ll << 31) &&
       threadIdx.x == 0)
     atomicOr(a.status, GVA_DEVERR_RANGE);
-  const TileSplit ts{tp[a.B], (int)gridDim.x};
+  // the tail pool needs one consumer warp per group (W == 1): a pool tile is a
+  // piece of its own
+  const TileSplit ts = make_split(tp[a.B], (int)gridDim.x, C::W == 1 ? a.pool_per_cta : 0);
+  const int n_pool = ts.pool();
   const CtaTiles rng{prefix, tp, a.B, ts.first(blockIdx.x), ts.first(blockIdx.x + 1), C::TT};
-  const bool has_work = !rng.empty();
+  const bool has_work = !rng.empty() || n_pool > 0;
   const int b_first = rng.first_seq();
+  // pool tile held by each stage (-1: the pool is empty, no data in the stage)
+  __shared__ int pool_tile[C::STAGES];
 
   // ------------------------------------------------------------------ producer
   // One thread issues every load of the CTA.  The cache is read once per step:
@@ -232,6 +240,35 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       issue(k);
       cur.next(rng);
     }
+    // Pool tiles, one per ticket once the static range is issued.  The next
+    // ticket is requested as soon as the current one is used, so the atomic's
+    // latency overlaps the wait for a free stage.  A stage that carries a pool
+    // tile names it in pool_tile[] (written before the arrive that completes the
+    // stage); -1 with a plain arrive (no bytes) tells the consumers the pool is
+    // empty.
+    if (prod_ok && n_pool > 0) {
+      int u = atomicAdd(a.pool_ctr, 1);
+      for (;; ++k) {
+        const int s = k % C::STAGES;
+        if (k >= C::STAGES &&
+            !mbar_wait(smem_u32(empty + s), ((k / C::STAGES) - 1) & 1, a.status)) {
+          prod_ok = false;
+          break;
+        }
+        if (u >= n_pool) {
+          pool_tile[s] = -1;
+          mbar_arrive(smem_u32(full + s));
+          ++k;
+          break;
+        }
+        const int v = ts.NS + u;
+        pool_tile[s] = v;
+        u = atomicAdd(a.pool_ctr, 1);
+        cur.b = seq_at(tp, a.B, v);
+        cur.t0 = (v - tp[cur.b]) * C::TT;
+        issue(k);
+      }
+    }
     (void)prod_ok;
     // Drain: do not leave while a copy into this CTA's shared memory is in flight.
     for (int kk = max(0, k - C::STAGES); kk < k; ++kk)
@@ -255,7 +292,11 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
   const int dq = C::D_H + a.d_r;
   // columns owned after the hi/lo merge: hcol, hcol+1 of this group.  Column c
   // is query c / hpr of the sequence's nq new tokens and head g*hpr + c % hpr.
+  // Fewer real columns than the configuration's (H/G * nq below 4, or 5..7 with
+  // 8): the rest carry a zero query and are never stored.
+  const int ncol = hpr * a.nq;
   const int hcol = (2 * t) & (C::HPG - 1);
+  const bool real0 = hcol < ncol, real1 = hcol + 1 < ncol;
   const int qi0 = hcol / hpr, qi1 = (hcol + 1) / hpr;   // differ only when H/G is odd
   const int phead0 = qi0 * H + g * hpr + hcol % hpr;
   const int phead1 = qi1 * H + g * hpr + (hcol + 1) % hpr;
@@ -265,13 +306,15 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
   bool ok = true;   // false once a bounded wait gave up: skip work, keep barrier order
 
   int k = 0;
-  for (int b = b_first; rng.reaches(b); ++b) {
-    int j0, j1;
-    if (!rng.piece(b, j0, j1)) continue;
-
-    // ---- query fragments (B operand of the score MMA): column n = gq
-    uint32_t qb[C::NT][C::KS][2];
-    uint32_t qr[C::NT][C::RS > 0 ? C::RS : 1][2];
+  // query fragments (B operand of the score MMA), column n = gq, of sequence q_seq
+  uint32_t qb[C::NT][C::KS][2];
+  uint32_t qr[C::NT][C::RS > 0 ? C::RS : 1][2];
+  int q_seq = -1;
+  // One piece: tokens [j0, j1) of sequence b, tiles k, k+1, ... of the ring;
+  // its partial state goes to `slot`.
+  auto run_piece = [&](const int b, const int j0, const int j1, const size_t slot) {
+    if (b != q_seq) {
+    q_seq = b;
 #pragma unroll
     for (int nt = 0; nt < C::NT; ++nt) {
       const int hl = C::HPG == 8 ? gq : (gq & 3);     // column within the group
@@ -281,7 +324,16 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       float wv[C::RS > 0 ? C::RS : 1][4];
       // absorbed fp32 query (pre-scaled), or the raw query in its storage type,
       // scaled here: GQA, and GVA with shared keys and values (M = I, d_r = 0)
-      if (!C::GQA && a.q_raw == nullptr) {
+      if (hl >= ncol) {   // padding column: zero query
+#pragma unroll
+        for (int ks = 0; ks < C::KS; ++ks)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) v[ks][e] = 0.f;
+#pragma unroll
+        for (int rs = 0; rs < (C::RS > 0 ? C::RS : 1); ++rs)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) wv[rs][e] = 0.f;
+      } else if (!C::GQA && a.q_raw == nullptr) {
         const float* qrow = a.q_abs + (((size_t)b * a.nq + vq) * H + head) * dq;
 #pragma unroll
         for (int ks = 0; ks < C::KS; ++ks) {
@@ -331,6 +383,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
         qr[nt][rs][0] = pack_bf16(part(wv[rs][0]), part(wv[rs][1]));
         qr[nt][rs][1] = pack_bf16(part(wv[rs][2]), part(wv[rs][3]));
       }
+    }
     }
 
     // O^T fragments: d rows x 8 columns.  With 8 columns per group the hi and lo
@@ -563,7 +616,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       }
       named_bar_sync(bar, nthr);   // scratch free for the next piece
     }
-    if (w != 0) continue;
+    if (w != 0) return;
     if constexpr (C::HPG == 4) {
 #pragma unroll
       for (int md = 0; md < C::KS; ++md)
@@ -571,23 +624,45 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
         for (int e = 0; e < 4; ++e) o[md][e] += __shfl_xor_sync(0xffffffffu, o[md][e], 2);
     }
     if (ok && (C::HPG == 8 || t < 2)) {
-      const size_t slot = (size_t)blockIdx.x + b;
       float* po0 = a.part_o + (slot * Hp + phead0) * C::D_H;
       float* po1 = a.part_o + (slot * Hp + phead1) * C::D_H;
 #pragma unroll
       for (int md = 0; md < C::KS; ++md) {
         const int d = md * 16 + gq;
-        po0[d] = o[md][0];
-        po1[d] = o[md][1];
-        po0[d + 8] = o[md][2];
-        po1[d + 8] = o[md][3];
+        if (real0) {
+          po0[d] = o[md][0];
+          po0[d + 8] = o[md][2];
+        }
+        if (real1) {
+          po1[d] = o[md][1];
+          po1[d + 8] = o[md][3];
+        }
       }
       if (gq == 0) {
-        a.part_ml[slot * Hp + phead0] = make_float2(m0, l0);
-        a.part_ml[slot * Hp + phead1] = make_float2(m1, l1);
+        if (real0) a.part_ml[slot * Hp + phead0] = make_float2(m0, l0);
+        if (real1) a.part_ml[slot * Hp + phead1] = make_float2(m1, l1);
       }
     }
     if (warp == 0 && lane == 0) trace_mark(a, 5);
+  };
+
+  // static range: its pieces land in slots cta + b
+  for (int b = b_first; rng.reaches(b); ++b) {
+    int j0, j1;
+    if (rng.piece(b, j0, j1)) run_piece(b, j0, j1, (size_t)blockIdx.x + b);
+  }
+  // pool tiles handed over by the producer, each a piece of one tile with its
+  // own slot, until the empty-pool mark
+  while (n_pool > 0 && ok) {
+    const int s = k % C::STAGES;
+    ok = mbar_wait(smem_u32(full + s), (k / C::STAGES) & 1, a.status);
+    if (!ok) break;
+    const int v = *static_cast<volatile int*>(pool_tile + s);
+    if (v < 0) break;
+    const int b = seq_at(tp, a.B, v);
+    const int j0 = (v - tp[b]) * C::TT;
+    run_piece(b, j0, min(j0 + C::TT, prefix[b + 1] - prefix[b]),
+              (size_t)gridDim.x + a.B + (size_t)(v - ts.NS));
   }
 }
 

@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(kSimtThreads)
   const int len_lane = (a.B <= 32 && tid < a.B) ? __ldg(a.seq_len + tid) : 0;
   if (scan_batch<kSimtTT>(a.seq_len, a.B, len_lane, prefix, tp, wtmp) >= (1ll << 31) && tid == 0)
     atomicOr(a.status, GVA_DEVERR_RANGE);
-  const TileSplit ts{tp[a.B], (int)gridDim.x};
+  const TileSplit ts = make_split(tp[a.B], (int)gridDim.x, 0);
   if (blockIdx.x == 0) write_meta(a, prefix, tp, ts);
   const CtaTiles rng{prefix, tp, a.B, ts.first(blockIdx.x), ts.first(blockIdx.x + 1), kSimtTT};
   if (rng.empty()) return;

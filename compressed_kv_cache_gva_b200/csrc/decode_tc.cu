@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
   if (scan_batch<C::TT>(a.seq_len, a.B, len_lane, prefix, tp, wtmp) >= (1ll << 31) &&
       threadIdx.x == 0)
     atomicOr(a.status, GVA_DEVERR_RANGE);
-  const TileSplit ts{tp[a.B], (int)gridDim.x};
+  const TileSplit ts = make_split(tp[a.B], (int)gridDim.x, 0);
   const CtaTiles rng{prefix, tp, a.B, ts.first(blockIdx.x), ts.first(blockIdx.x + 1), C::TT};
   const bool has_work = !rng.empty();
   const int b_first = rng.first_seq();

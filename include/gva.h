@@ -23,6 +23,12 @@
  *   - All work is enqueued asynchronously on `stream` (a cudaStream_t passed as
  *     void*, NULL = legacy default stream).  Outputs are valid once the stream has
  *     reached that point.
+ *   - Kernels are launched with programmatic dependent launch and let the next
+ *     kernel on the stream start early (the combine and the first kernel of a
+ *     fused step do so at entry).  A kernel of the caller's that is itself
+ *     launched with programmatic stream serialization right after a call here
+ *     must execute griddepcontrol.wait (cudaGridDependencySynchronize) before it
+ *     reads that call's outputs; normally launched kernels need nothing.
  *   - Host-side validation happens before anything is launched; a non-OK status
  *     means nothing was enqueued.  gva_last_error() returns a one-line reason for
  *     the last non-OK status of the calling thread.  GVA_ERR_CUDA reports a launch
@@ -131,16 +137,18 @@ gva_status_t gva_append_cache(const gva_shape_t* shape, int32_t N, const void* v
  * device's SM count) when the total cached tokens never exceed max_total_tokens.
  * Returns 0 for an invalid shape.
  *
- * Workspace contract: the first 4 bytes are a device status word.  Zero it once
- * (e.g. cudaMemsetAsync of the whole buffer) before first use; the library never
- * clears it.  After a decode it holds 0, or a nonzero GVA_DEVERR_* bit mask if a
- * kernel met an inconsistent input (a sequence reaching outside [0, num_slots))
- * or gave up a bounded wait.  The rest of the buffer is overwritten every call.
+ * Workspace contract: the first 4 bytes are a device status word, the next 4 a
+ * work counter of the split kernel.  Zero the buffer once (e.g. cudaMemsetAsync
+ * of the whole buffer) before first use; the library never clears the status
+ * word, and every decode leaves the counter at 0 again.  After a decode the
+ * status holds 0, or a nonzero GVA_DEVERR_* bit mask if a kernel met an
+ * inconsistent input (a sequence reaching outside [0, num_slots)) or gave up a
+ * bounded wait.  The rest of the buffer is overwritten every call.
  */
 size_t gva_decode_workspace_size(const gva_shape_t* shape, int64_t max_total_tokens);
 
 #define GVA_DEVERR_RANGE 1   /* some sequence's slots leave [0, num_slots); those rows read as 0 */
-#define GVA_DEVERR_WAIT 2    /* a pipeline wait hit its iteration limit; outputs invalid */
+#define GVA_DEVERR_WAIT 2    /* a pipeline wait hit its poll or time limit; outputs invalid */
 
 /*
  * gva_decode_attention — one GVA decode step over a (possibly ragged) batch,
@@ -270,7 +278,7 @@ gva_status_t gva_decode_step(const gva_shape_t* shape, const void* q, const void
  *   Other arguments as gva_decode_attention.  n_query = 1 is gva_decode_attention.
  *
  * Two kernels, by the number of query columns per value group, (H/G)*n_query:
- *  - 4 or 8 (speculative blocks): the split-KV decode kernel (mma.sync), the
+ *  - up to 8 (speculative blocks): the split-KV decode kernel (mma.sync), the
  *    columns sharing each tile, then the combine; bf16 cache, d_h in {64, 128};
  *  - more than 8 (chunked prefill, long drafts): the tcgen05 kernel, one CTA per
  *    128 query rows (token x head) of a group, scores and outputs accumulated in

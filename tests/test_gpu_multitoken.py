@@ -45,7 +45,7 @@ def oracle_multi(di, q, qpos):
 
 
 CASES = [
-    # (workload, n_query, lengths): H/G * n_query must be 4 or 8
+    # (workload, n_query, lengths): H/G * n_query columns per group, at most 8
     ("350m_b8_t4096", 2, [1500, 2, 3001, 17, 64, 65, 1, 700]),
     ("dr24_b4_t32768", 2, [4100, 33, 2]),
     ("d128_b1_t131072", 2, [2900, 130]),          # H/G = 4
@@ -53,6 +53,8 @@ CASES = [
     ("mha_h8_g8", 4, [1000, 3, 4, 260]),          # H/G = 1: a thread's two columns are two queries
     ("h8_g4", 4, [777, 9]),                       # H/G = 2, 8 columns
     ("h8_g4", 2, [777, 9]),                       # H/G = 2, 4 columns
+    ("mha_h8_g8", 3, [500, 2, 40]),               # 3 columns, one zero-query padding column
+    ("h8_g4", 3, [777, 9, 64]),                   # 6 columns, two padding columns
 ]
 
 EXTRA = {
