@@ -5,6 +5,8 @@
 //   lse = (m* + log2 L) * ln 2  (natural log of sum_j exp(s_j)).
 // The merge order is fixed by piece index, so results do not depend on which CTA
 // finished first.
+#include <type_traits>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -12,7 +14,12 @@ namespace gva {
 
 constexpr int kCombineScanMaxB = 64;   // batches up to this size find their pieces
                                         // from the lengths before waiting
-constexpr int kCombinePieces = 8;       // pieces per thread requested at once
+// Target pieces per thread of the combine (loads requested at once); the launcher
+// picks the block size from it and the expected pieces per sequence.
+#ifndef GVA_COMBINE_PIECES
+#define GVA_COMBINE_PIECES 8
+#endif
+constexpr int kCombinePieces = GVA_COMBINE_PIECES;
 
 // grid (B, H, ceil(d_h / 32)); block = 32 output columns x PG piece groups.
 // Thread (pg, lane) merges pieces pg, pg+PG, ... of column d = 32*z + lane with
@@ -21,7 +28,7 @@ constexpr int kCombinePieces = 8;       // pieces per thread requested at once
 // the piece range of sequence b is recomputed from the lengths (caller input)
 // before waiting on the split kernel, so that after the wait only the partials
 // are read.
-template <typename TO>
+template <typename TO, int PPT>
 __global__ void __launch_bounds__(1024)
     combine_kernel(const DecodeArgs a, TO* __restrict__ out, float* __restrict__ lse) {
   __shared__ float sm_m[32][33], sm_l[32][33], sm_o[32][33];
@@ -92,11 +99,11 @@ __global__ void __launch_bounds__(1024)
   const float* po = a.part_o + ((size_t)meta.x * H + h) * d_h + (col ? d : 0);
   const size_t mstride = H, ostride = (size_t)H * d_h;
   float m = -INFINITY, l = 0.f, o = 0.f;
-  for (int c0 = pg; c0 < n; c0 += kCombinePieces * npg) {
-    float2 e[kCombinePieces];
-    float x[kCombinePieces];
+  for (int c0 = pg; c0 < n; c0 += PPT * npg) {
+    float2 e[PPT];
+    float x[PPT];
 #pragma unroll
-    for (int u = 0; u < kCombinePieces; ++u) {
+    for (int u = 0; u < PPT; ++u) {
       const int c = c0 + u * npg;
       if (c < n) {
         const long long sl = c < sc ? c : (long long)c + pool_shift;   // relative to meta.x
@@ -105,7 +112,7 @@ __global__ void __launch_bounds__(1024)
       }
     }
 #pragma unroll
-    for (int u = 0; u < kCombinePieces; ++u) {
+    for (int u = 0; u < PPT; ++u) {
       if (c0 + u * npg >= n) break;
       if (e[u].x == -INFINITY) continue;          // piece past this query's causal limit
       const float mn = fmaxf(m, e[u].x);
@@ -154,10 +161,23 @@ cudaError_t launch_combine(const gva_shape_t& sh, const DecodeArgs& a, void* out
   const int per_seq = a.grid * (1 + a.pool_per_cta) / (sh.B > 0 ? sh.B : 1) + 2;
   int npg = (per_seq + kCombinePieces - 1) / kCombinePieces;
   npg = npg < 1 ? 1 : (npg > 32 ? 32 : npg);
-  if (sh.out_dtype == GVA_BF16)
-    return launch_pdl(combine_kernel<__nv_bfloat16>, grid, dim3(32 * npg), 0, st, a,
-                      (__nv_bfloat16*)out, lse);
-  return launch_pdl(combine_kernel<float>, grid, dim3(32 * npg), 0, st, a, (float*)out, lse);
+  // loads per thread: enough that one round covers the expected pieces when the
+  // block is at its 1024-thread limit (a second round costs a full L2 latency)
+  const int need = (per_seq + npg - 1) / npg;
+  const int ppt = need <= kCombinePieces ? kCombinePieces : 16;   // 32 would spill at 1024 threads
+  auto go = [&](auto ppt_c, auto* o) {
+    constexpr int K = decltype(ppt_c)::value;
+    using TO = std::remove_pointer_t<decltype(o)>;
+    return launch_pdl(combine_kernel<TO, K>, grid, dim3(32 * npg), 0, st, a, o, lse);
+  };
+  using K8 = std::integral_constant<int, kCombinePieces>;
+  using K16 = std::integral_constant<int, (kCombinePieces > 16 ? kCombinePieces : 16)>;
+  if (sh.out_dtype == GVA_BF16) {
+    auto* o = (__nv_bfloat16*)out;
+    return ppt <= kCombinePieces ? go(K8{}, o) : go(K16{}, o);
+  }
+  auto* o = (float*)out;
+  return ppt <= kCombinePieces ? go(K8{}, o) : go(K16{}, o);
 }
 
 // Merge of R normalised attention states of the same queries over disjoint parts

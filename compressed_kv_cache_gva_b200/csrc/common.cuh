@@ -35,10 +35,12 @@ constexpr unsigned long long kWaitNs = GVA_WAIT_NS;
 // Tail pool of the split (see TileSplit): when a batch has at least
 // kPoolMinTilesPerCta tiles per CTA, its last kPoolTilesPerCta * grid tiles are
 // not assigned statically; CTAs that finish their static range take them one at
-// a time.  0 disables the pool.
+// a time.  0 (the default) disables the pool: measured on B200 it made the long
+// decodes slower, because all pool partials belong to the batch's last sequences
+// and their combine blocks then merge hundreds of pieces each.
 // ---------------------------------------------------------------------------
 #ifndef GVA_POOL_TILES_PER_CTA
-#define GVA_POOL_TILES_PER_CTA 1
+#define GVA_POOL_TILES_PER_CTA 0
 #endif
 constexpr int kPoolTilesPerCta = GVA_POOL_TILES_PER_CTA;
 constexpr int kPoolMinTilesPerCta = 4;

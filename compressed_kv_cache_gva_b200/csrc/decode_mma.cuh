@@ -27,7 +27,12 @@
 
 namespace gva {
 
-template <int D_H_, int NG_, int HPG_, int DRP_, bool GQA_, int W_ = 0>
+#ifndef GVA_ROW_PARTS   // consumer warps per group splitting every tile's rows (d_h = 64, G <= 4)
+#define GVA_ROW_PARTS 1
+#endif
+
+template <int D_H_, int NG_, int HPG_, int DRP_, bool GQA_, int W_ = 0,
+          int P_ = (D_H_ == 64 && NG_ <= 4) ? GVA_ROW_PARTS : 1>
 struct MmaCfg {
   static constexpr int D_H = D_H_, NG = NG_, HPG = HPG_, DRP = GQA_ ? 0 : DRP_;
   static constexpr bool GQA = GQA_;
@@ -50,6 +55,11 @@ struct MmaCfg {
   // per group is fastest for every workload here (a second warp per group adds the
   // end-of-piece merge and contends for the same SM resources), so 0 means 1.
   static constexpr int W = W_ > 0 ? W_ : 1;
+  // P warps per group can instead split every tile's 16-row blocks between them
+  // (all P consume each tile; their states merge at the end of a piece), which
+  // shortens each tile's dependent MMA/softmax chain.  W and P do not combine.
+  static constexpr int P = P_ > 0 ? P_ : 1;
+  static constexpr int GW = W * P;                    // consumer warps per group
   static constexpr int STAGES_RAW = GVA_PIPE_BYTES / STAGE;
   static constexpr int STAGES_CLAMPED = STAGES_RAW < 2 ? 2 : (STAGES_RAW > 12 ? 12 : STAGES_RAW);
   // A multiple of W: tile k lives in stage k % STAGES and is consumed by warp
@@ -58,20 +68,24 @@ struct MmaCfg {
   // count a warp could wait for phase p+2 while the stage is still in phase p+1,
   // and the parity test would pass on stale data.)
   static constexpr int STAGES = STAGES_CLAMPED / W * W < W ? W : STAGES_CLAMPED / W * W;
+#ifndef GVA_RAMP_TILES   // tiles requested before the first one has landed (0: the whole ring)
+#define GVA_RAMP_TILES 0
+#endif
+  static constexpr int RAMP = GVA_RAMP_TILES > 0 && GVA_RAMP_TILES < STAGES ? GVA_RAMP_TILES : 0;
   static constexpr int PIPE = STAGES * STAGE;
   static constexpr uint32_t TX = XB + VB + KRB;       // bytes TMA delivers per stage
   static constexpr int MT = TT / 16;                  // 16-token m-tiles per tile
-  static constexpr int MW = MT;                       // m-tiles per consumer warp and tile
-  static constexpr int NCW = NG * W;                  // consumer warps
+  static constexpr int MW = MT / P;                   // m-tiles per consumer warp and tile
+  static constexpr int NCW = NG * GW;                 // consumer warps
   static constexpr int THREADS = (NCW + 1) * 32;
   static constexpr int NT = HPG == 8 ? 2 : 1;         // 8-column MMA tiles
   static constexpr int KS = D_H / 16;                 // content k-steps (= d m-tiles)
   static constexpr int RS = DRP / 16;                 // positional k-steps
-  // end-of-piece merge of the W warps of a group: (m, l) per warp and lane quad,
-  // and the output fragments of warps 1..W-1
-  static constexpr int MERGE_ML = W * 4 * 4;                    // floats per group
-  static constexpr int MERGE_O = (W - 1) * 32 * KS * 4;        // floats per group
-  static constexpr int MERGE = W > 1 ? NG * (MERGE_ML + MERGE_O) * 4 : 0;  // bytes
+  // end-of-piece merge of the GW warps of a group: (m, l) per warp and lane quad,
+  // and the output fragments of warps 1..GW-1
+  static constexpr int MERGE_ML = GW * 4 * 4;                   // floats per group
+  static constexpr int MERGE_O = (GW - 1) * 32 * KS * 4;       // floats per group
+  static constexpr int MERGE = GW > 1 ? NG * (MERGE_ML + MERGE_O) * 4 : 0;  // bytes
   static constexpr int KR_SW = DRP * 2;               // swizzle span of the k_rope box
   // resident CTAs per SM the register budget is sized for.  Two CTAs of 9 warps
   // leave 96 registers a thread; 8 columns of d_h = 128 keep ~100 values live in
@@ -80,6 +94,8 @@ struct MmaCfg {
   static constexpr int MINB = (NCW >= 8 && HPG == 8 && D_H == 128) ? 1 : 2;
   static_assert(HPG == 4 || HPG == 8, "heads per group");
   static_assert(STAGES % W == 0, "each stage must belong to one warp of a group");
+  static_assert(W == 1 || P == 1, "round robin over tiles or rows split, not both");
+  static_assert(MT % P == 0, "row parts must divide the tile's 16-row blocks");
   static_assert(D_H % 64 == 0, "d_h");
   static_assert(DRP == 0 || DRP == 16 || DRP == 32, "padded d_r");
 
@@ -120,7 +136,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(smem_u32(full + s), 1);
-      mbar_init(smem_u32(empty + s), C::NG);   // one warp per group consumes a tile
+      mbar_init(smem_u32(empty + s), C::NG * C::P);   // the warps of a group that read a tile
     }
     fence_barrier_init();
   }
@@ -140,8 +156,9 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
     atomicOr(a.status, GVA_DEVERR_RANGE);
   // the tail pool needs one consumer warp per group (W == 1): a pool tile is a
   // piece of its own
-  const TileSplit ts = make_split(tp[a.B], (int)gridDim.x, C::W == 1 ? a.pool_per_cta : 0);
-  const int n_pool = ts.pool();
+  const TileSplit ts = make_split(tp[a.B], (int)gridDim.x,
+                                  (kPoolTilesPerCta > 0 && C::W == 1) ? a.pool_per_cta : 0);
+  const int n_pool = kPoolTilesPerCta > 0 ? ts.pool() : 0;   // compiled out when disabled
   const CtaTiles rng{prefix, tp, a.B, ts.first(blockIdx.x), ts.first(blockIdx.x + 1), C::TT};
   const bool has_work = !rng.empty() || n_pool > 0;
   const int b_first = rng.first_seq();
@@ -237,6 +254,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
         prod_ok = false;
         break;
       }
+      // ramp: the rest of the ring is requested once the first tile has landed
+      if (C::RAMP > 0 && k == C::RAMP) mbar_wait(smem_u32(full), 0, a.status);
       issue(k);
       cur.next(rng);
     }
@@ -280,7 +299,11 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
   // warp = g * W + w: group g, tiles w, w+W, w+2W, ... of this CTA (round robin,
   // so W tiles per group are in flight); the W running states are merged at the
   // end of every piece
-  const int g = warp / C::W, w = warp % C::W;
+  // warp = g * GW + wi: group g; with W > 1 warp wi takes tiles wi, wi+W, ...,
+  // with P > 1 it takes rows [wi*16*MW, (wi+1)*16*MW) of every tile
+  const int g = warp / C::GW, wi = warp % C::GW;
+  const int w = C::W > 1 ? wi : 0;
+  const int r_lo = C::P > 1 ? wi * C::MW * 16 : 0, r_hi = r_lo + C::MW * 16;   // this warp's rows
   const int t = lane & 3, gq = lane >> 2;
   const int mi = lane >> 3, r8 = lane & 7;
   // ldmatrix row/chunk owned by this lane (see the fragment layouts of m16n8k16)
@@ -418,7 +441,6 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       uint8_t* st = pipe + s * C::STAGE;
       uint8_t* xg = st + g * C::CB * C::BOX;
       uint8_t* vg = C::GQA ? st + C::XB + g * C::CB * C::BOX : xg;
-      const int r_lo = 0, r_hi = C::TT;   // this warp's rows: the whole tile
       const bool ragged = nvalid < r_hi;
       if (ragged) {
         // rows past the sequence may hold anything (even NaN): zero this warp's
@@ -436,7 +458,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       float sc[C::MW][4];
 #pragma unroll
       for (int mm = 0; mm < C::MW; ++mm) {
-        const int arow = a_row + mm * 16;
+        const int arow = a_row + r_lo + mm * 16;
         float acc[2][C::NT][4];
 #pragma unroll
         for (int c2 = 0; c2 < 2; ++c2)
@@ -481,7 +503,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       for (int mm = 0; mm < C::MW; ++mm)
 #pragma unroll
         for (int md = 0; md < C::KS; ++md)
-          ldsm_x4_t(vg_u + (md >> 2) * C::BOX + (v_tok + mm * 16) * 128 +
+          ldsm_x4_t(vg_u + (md >> 2) * C::BOX + (v_tok + r_lo + mm * 16) * 128 +
                         ((((md & 3) * 2 + v_dc) ^ r8) << 4),
                     vf[mm][md][0], vf[mm][md][1], vf[mm][md][2], vf[mm][md][3]);
 
@@ -559,17 +581,17 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       l0 += __shfl_xor_sync(0xffffffffu, l0, off);
       l1 += __shfl_xor_sync(0xffffffffu, l1, off);
     }
-    if constexpr (C::W > 1) {
-      // merge the W warps of this group: common max, rescale, sum through smem
-      const int bar = 1 + g, nthr = C::W * 32;
+    if constexpr (C::GW > 1) {
+      // merge the GW warps of this group: common max, rescale, sum through smem
+      const int bar = 1 + g, nthr = C::GW * 32;
       if (gq == 0) {
-        float* e = mg_ml + (w * 4 + t) * 4;
+        float* e = mg_ml + (wi * 4 + t) * 4;
         e[0] = m0; e[1] = m1; e[2] = l0; e[3] = l1;
       }
       named_bar_sync(bar, nthr);
       float M0 = -INFINITY, M1 = -INFINITY;
 #pragma unroll
-      for (int u = 0; u < C::W; ++u) {
+      for (int u = 0; u < C::GW; ++u) {
         M0 = fmaxf(M0, mg_ml[(u * 4 + t) * 4 + 0]);
         M1 = fmaxf(M1, mg_ml[(u * 4 + t) * 4 + 1]);
       }
@@ -578,7 +600,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       const float Ms0 = M0 == -INFINITY ? 0.f : M0, Ms1 = M1 == -INFINITY ? 0.f : M1;
       float L0 = 0.f, L1 = 0.f;
 #pragma unroll
-      for (int u = 0; u < C::W; ++u) {
+      for (int u = 0; u < C::GW; ++u) {
         const float* e = mg_ml + (u * 4 + t) * 4;
         L0 += e[2] * ex2(e[0] - Ms0);
         L1 += e[3] * ex2(e[1] - Ms1);
@@ -592,17 +614,17 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
         o[md][3] *= f1;
       }
       m0 = M0; m1 = M1; l0 = L0; l1 = L1;
-      if (w > 0) {
-        float* dst = mg_o + ((w - 1) * 32 + lane) * (C::KS * 4);
+      if (wi > 0) {
+        float* dst = mg_o + ((wi - 1) * 32 + lane) * (C::KS * 4);
 #pragma unroll
         for (int md = 0; md < C::KS; ++md)
           *reinterpret_cast<float4*>(dst + md * 4) =
               make_float4(o[md][0], o[md][1], o[md][2], o[md][3]);
       }
       named_bar_sync(bar, nthr);
-      if (w == 0) {
+      if (wi == 0) {
 #pragma unroll
-        for (int u = 1; u < C::W; ++u) {
+        for (int u = 1; u < C::GW; ++u) {
           const float* src = mg_o + ((u - 1) * 32 + lane) * (C::KS * 4);
 #pragma unroll
           for (int md = 0; md < C::KS; ++md) {
@@ -616,7 +638,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       }
       named_bar_sync(bar, nthr);   // scratch free for the next piece
     }
-    if (w != 0) return;
+    if (wi != 0) return;
     if constexpr (C::HPG == 4) {
 #pragma unroll
       for (int md = 0; md < C::KS; ++md)

@@ -15,7 +15,7 @@ the two score terms.  The GPU path instead folds M_h into the query; the review'
 "How it works" section (어떻게 동작하나) states that the two routes give the same
 score exactly, so agreement between them is the parity claim.
 
-Readings where the pages are silent (each is also listed in the design notes):
+Readings where the pages are silent:
   * softmax scale 1/sqrt(d_n + d_r);
   * RoPE pairs dimension i with i + d_r/2 ("rotate half"), frequency
     theta_i = base^(-2i/d_r), angle = position * theta_i evaluated in float64;
@@ -25,7 +25,9 @@ Readings where the pages are silent (each is also listed in the design notes):
     the query's own position is an explicit input;
   * an empty sequence (L_b = 0) gives a zero output and lse = -inf;
   * the stored positional key is the exact rotation rounded once to the cache
-    type (round to nearest, ties to even).
+    type (round to nearest, ties to even);
+  * the matched GQA baseline rotates its whole key (and query) of width d_h the
+    same way, pair i with i + d_h/2.
 
 Every function is plain numpy in float64: per (sequence, head) loops around
 library matmuls, no blocking, no fusion, no reordering beyond the definitions.
