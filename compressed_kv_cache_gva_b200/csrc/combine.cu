@@ -16,8 +16,8 @@ constexpr int kCombineScanMaxB = 64;   // batches up to this size find their pie
                                         // from the lengths before waiting
 // Target pieces per thread of the combine (loads requested at once); the launcher
 // picks the block size from it and the expected pieces per sequence.
-#ifndef GVA_COMBINE_PIECES
-#define GVA_COMBINE_PIECES 8
+#ifndef GVA_COMBINE_PIECES   // measured on B200: 4 beats 8 on every decode workload here
+#define GVA_COMBINE_PIECES 4
 #endif
 constexpr int kCombinePieces = GVA_COMBINE_PIECES;
 
@@ -165,6 +165,7 @@ cudaError_t launch_combine(const gva_shape_t& sh, const DecodeArgs& a, void* out
   // block is at its 1024-thread limit (a second round costs a full L2 latency)
   const int need = (per_seq + npg - 1) / npg;
   const int ppt = need <= kCombinePieces ? kCombinePieces : 16;   // 32 would spill at 1024 threads
+  static_assert(kCombinePieces <= 16, "pieces per thread");
   auto go = [&](auto ppt_c, auto* o) {
     constexpr int K = decltype(ppt_c)::value;
     using TO = std::remove_pointer_t<decltype(o)>;
