@@ -60,8 +60,11 @@ struct MmaCfg {
   // shortens each tile's dependent MMA/softmax chain.  W and P do not combine.
   static constexpr int P = P_ > 0 ? P_ : 1;
   static constexpr int GW = W * P;                    // consumer warps per group
-#ifndef GVA_PIPE_BYTES_WIDE   // ring budget of the 33 KB tiles of eight 128-wide groups
-#define GVA_PIPE_BYTES_WIDE GVA_PIPE_BYTES
+// Ring budget of the 33 KB tiles of eight 128-wide groups: 3 stages instead of
+// the 2 that GVA_PIPE_BYTES holds (measured: 131k-token decode 52.2 -> 50.2 us,
+// other shapes unaffected); two CTAs per SM still fit.
+#ifndef GVA_PIPE_BYTES_WIDE
+#define GVA_PIPE_BYTES_WIDE (108 * 1024)
 #endif
   static constexpr int PIPE_BUDGET =
       (!GQA && D_H == 128 && NG == 8) ? GVA_PIPE_BYTES_WIDE : GVA_PIPE_BYTES;
@@ -97,14 +100,6 @@ struct MmaCfg {
   static constexpr int MERGE_O = (GW - 1) * 32 * KS * 4;       // floats per group
   static constexpr int MERGE = GW > 1 ? NG * (MERGE_ML + MERGE_O) * 4 : 0;  // bytes
   static constexpr int KR_SW = DRP * 2;               // swizzle span of the k_rope box
-#ifndef GVA_QUERY_STAGE   // stage the next piece's query rows in shared memory (cp.async)
-#define GVA_QUERY_STAGE 0
-#endif
-  // per consumer warp: the HPG query rows of the next piece (fp32 absorbed rows of
-  // D_H + d_r <= D_H + DRP values, or raw rows of D_H values)
-  static constexpr int QROW = (D_H + DRP) * 4;                 // bytes per staged row
-  static constexpr int QST = GVA_QUERY_STAGE ? HPG * QROW : 0; // bytes per warp
-  static constexpr int QSTAGE = NCW * QST;
   // resident CTAs per SM the register budget is sized for.  Two CTAs of 9 warps
   // leave 96 registers a thread; 8 columns of d_h = 128 keep ~100 values live in
   // the consumer (query fragments, O^T accumulators, V^T fragments), so that
@@ -118,7 +113,7 @@ struct MmaCfg {
   static_assert(DRP == 0 || DRP == 16 || DRP == 32, "padded d_r");
 
   static size_t smem_bytes(int B) {
-    return 1024 + PIPE + MERGE + QSTAGE + 16 * STAGES + 3 * sizeof(int) * (B + 1) + 16 +
+    return 1024 + PIPE + MERGE + 16 * STAGES + 3 * sizeof(int) * (B + 1) + 16 +
            sizeof(long long) * 33;
   }
 };
@@ -132,8 +127,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
   uint8_t* pipe = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
                                              ~uintptr_t(1023));
   float* merge = reinterpret_cast<float*>(pipe + C::PIPE);
-  uint8_t* qstage = pipe + C::PIPE + C::MERGE;
-  uint64_t* full = reinterpret_cast<uint64_t*>(pipe + C::PIPE + C::MERGE + C::QSTAGE);
+  uint64_t* full = reinterpret_cast<uint64_t*>(pipe + C::PIPE + C::MERGE);
   uint64_t* empty = full + C::STAGES;
   int* prefix = reinterpret_cast<int*>(empty + C::STAGES);
   int* offs = prefix + a.B + 1;
@@ -348,36 +342,6 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
   float* mg_o = mg_ml + C::MERGE_ML;
   bool ok = true;   // false once a bounded wait gave up: skip work, keep barrier order
 
-#if GVA_QUERY_STAGE
-  // The query rows of a piece reach the warp through its staging area: the copy of
-  // the next piece's rows starts when a piece starts, so a CTA whose tiles cross
-  // into another sequence does not wait for a query load at the crossing.
-  const bool absq = !C::GQA && a.q_raw == nullptr;
-  const int qrow_bytes = absq ? dq * 4 : C::D_H * (a.q_bf16 ? 2 : 4);   // a multiple of 8
-  const char* qbase = absq ? reinterpret_cast<const char*>(a.q_abs)
-                           : reinterpret_cast<const char*>(a.q_raw);
-  uint8_t* qst = qstage + warp * C::QST;
-  auto stage_query = [&](int bs) {   // real columns only (padding columns have no row)
-    const int ch = qrow_bytes / 8;
-#pragma unroll 1
-    for (int i = lane; i < ncol * ch; i += 32) {
-      const int hl = i / ch, c = i - hl * ch;
-      const int vq = hl / hpr, head = g * hpr + hl % hpr;
-      cp_async_8(smem_u32(qst + hl * C::QROW + c * 8),
-                 qbase + (((size_t)bs * a.nq + vq) * H + head) * qrow_bytes + c * 8);
-    }
-    cp_async_commit();
-  };
-  auto next_piece = [&](int from) {   // next sequence with tiles in this CTA's static range
-    int x0, x1;
-    while (rng.reaches(from) && !rng.piece(from, x0, x1)) ++from;
-    return from;
-  };
-  {
-    const int b0 = next_piece(b_first);
-    if (rng.reaches(b0)) stage_query(b0);
-  }
-#endif
   int k = 0;
   // query fragments (B operand of the score MMA), column n = gq, of sequence q_seq
   uint32_t qb[C::NT][C::KS][2];
@@ -388,10 +352,6 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
   auto run_piece = [&](const int b, const int j0, const int j1, const size_t slot) {
     if (b != q_seq) {
     q_seq = b;
-#if GVA_QUERY_STAGE
-    cp_async_wait_all();
-    __syncwarp();
-#endif
 #pragma unroll
     for (int nt = 0; nt < C::NT; ++nt) {
       const int hl = C::HPG == 8 ? gq : (gq & 3);     // column within the group
@@ -411,11 +371,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
 #pragma unroll
           for (int e = 0; e < 4; ++e) wv[rs][e] = 0.f;
       } else if (!C::GQA && a.q_raw == nullptr) {
-#if GVA_QUERY_STAGE
-        const float* qrow = reinterpret_cast<const float*>(qst + hl * C::QROW);
-#else
         const float* qrow = a.q_abs + (((size_t)b * a.nq + vq) * H + head) * dq;
-#endif
 #pragma unroll
         for (int ks = 0; ks < C::KS; ++ks) {
           const int k0 = ks * 16 + 2 * t;
@@ -435,12 +391,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
           wv[rs][3] = k0 + 9 < a.d_r ? qrow[C::D_H + k0 + 9] : 0.f;
         }
       } else {
-#if GVA_QUERY_STAGE
-        const void* rawrow = qst + hl * C::QROW;
-#else
         const void* rawrow = reinterpret_cast<const char*>(a.q_raw) +
             (((size_t)b * a.nq + vq) * H + head) * C::D_H * (a.q_bf16 ? 2 : 4);
-#endif
 #pragma unroll
         for (int ks = 0; ks < C::KS; ++ks) {
           const int k0 = ks * 16 + 2 * t;
@@ -470,13 +422,6 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
         qr[nt][rs][1] = pack_bf16(part(wv[rs][2]), part(wv[rs][3]));
       }
     }
-#if GVA_QUERY_STAGE
-    __syncwarp();   // every lane has read the rows: start the next piece's copy
-    {
-      const int bn = next_piece(b + 1);
-      if (rng.reaches(bn)) stage_query(bn);
-    }
-#endif
     }
 
     // O^T fragments: d rows x 8 columns.  With 8 columns per group the hi and lo
