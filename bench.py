@@ -667,17 +667,20 @@ def run_ours(args, rank, world, local):
     return res, st.di
 
 
-def time_e2e_pipelined(st, parts, h_stage, nb, view, K, dev, timer):
-    """End-to-end steps with double-buffered host<->device copies, ms per step.
+E2E_BUFFERS = 2   # staging / output buffers of the pipelined end-to-end loop
 
-    Step i copies its inputs (one pinned host buffer -> device staging buffer i % 2)
-    on one copy stream, runs gva_decode_step on the compute stream once that copy
-    has landed, and copies its output (device buffer i % 2 -> pinned host buffer
-    i % 2) on a second copy stream.  A staging buffer is refilled only after the
-    step that read it has finished, and an output buffer is rewritten only after
-    its previous copy-out has finished, so every step reads its own inputs and every
-    output reaches the host."""
-    NBUF = 2
+
+def time_e2e_pipelined(st, parts, h_stage, nb, view, K, dev, timer, nbuf=None):
+    """End-to-end steps with multi-buffered host<->device copies, ms per step.
+
+    Step i copies its inputs (one pinned host buffer -> device staging buffer
+    i % NBUF) on one copy stream, runs gva_decode_step on the compute stream once
+    that copy has landed, and copies its output (device buffer i % NBUF -> pinned
+    host buffer i % NBUF) on a second copy stream.  A staging buffer is refilled
+    only after the step that read it has finished, and an output buffer is
+    rewritten only after its previous copy-out has finished, so every step reads
+    its own inputs and every output reaches the host."""
+    NBUF = nbuf or E2E_BUFFERS
     B, H, d_h, R = st.B, st.wl.H, st.wl.d_h, st.R
     d_st = [torch.zeros(nb, dtype=torch.uint8, device=dev) for _ in range(NBUF)]
     o_dev = [torch.empty(B, H, d_h, dtype=torch.float32, device=dev) for _ in range(NBUF)]

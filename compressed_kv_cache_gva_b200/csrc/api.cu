@@ -242,10 +242,14 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
     a.tile = gva::mma_tile(sh, gqa);
     const int tt = a.tile;
     const int row = sh.G * sh.d_h;
+    // value (and GQA key) boxes: 64 columns with a 128-byte swizzle, or one
+    // 32-column group with a 64-byte swizzle for d_h = 32
+    const int vw = sh.d_h < 64 ? sh.d_h : 64;
+    const CUtensorMapSwizzle vsw = vw == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     CUtensorMap tx{}, tv{}, tk{};
-    if ((s = encode_2d(&tx, X, num_slots, row, row, tt, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != GVA_OK) return s;
+    if ((s = encode_2d(&tx, X, num_slots, row, row, tt, vw, vsw)) != GVA_OK) return s;
     tv = tx;
-    if (gqa && (s = encode_2d(&tv, Vv, num_slots, row, row, tt, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != GVA_OK)
+    if (gqa && (s = encode_2d(&tv, Vv, num_slots, row, row, tt, vw, vsw)) != GVA_OK)
       return s;
     tk = tx;
     if (!gqa && sh.d_r > 0) {

@@ -32,12 +32,16 @@ bool dispatch(const gva_shape_t& sh, bool gqa, F&& f) {
 #define GVA_CASES_NG(DH, HPG, DRP, GQ) \
   GVA_CASE(DH, 2, HPG, DRP, GQ) GVA_CASE(DH, 4, HPG, DRP, GQ) GVA_CASE(DH, 8, HPG, DRP, GQ)
 #define GVA_CASES_HPG(DH, DRP, GQ) GVA_CASES_NG(DH, 4, DRP, GQ) GVA_CASES_NG(DH, 8, DRP, GQ)
+  GVA_CASES_HPG(32, 0, false)
+  GVA_CASES_HPG(32, 16, false)
+  GVA_CASES_HPG(32, 32, false)
   GVA_CASES_HPG(64, 0, false)
   GVA_CASES_HPG(64, 16, false)
   GVA_CASES_HPG(64, 32, false)
   GVA_CASES_HPG(128, 0, false)
   GVA_CASES_HPG(128, 16, false)
   GVA_CASES_HPG(128, 32, false)
+  GVA_CASES_HPG(32, 0, true)
   GVA_CASES_HPG(64, 0, true)
   GVA_CASES_HPG(128, 0, true)
 #undef GVA_CASES_HPG

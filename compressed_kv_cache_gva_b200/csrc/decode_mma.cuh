@@ -42,8 +42,13 @@ struct MmaCfg {
 #endif
   static constexpr int TT_RAW = (GQA ? 2 * GVA_TILE_BYTES : GVA_TILE_BYTES) / ROW_BYTES;
   static constexpr int TT = TT_RAW >= 64 ? 64 : (TT_RAW >= 32 ? 32 : 16);   // tokens per tile
-  static constexpr int CB = D_H / 64;                 // 64-column boxes per group
-  static constexpr int BOX = TT * 128;                // bytes of one [TT x 64] bf16 box
+  // A group's values arrive as boxes of VW columns (64, or 32 for d_h = 32), one
+  // VROW-byte row per token, swizzled over VROW bytes by the TMA
+  static constexpr int VW = D_H < 64 ? D_H : 64;      // columns per box
+  static constexpr int VROW = VW * 2;                 // bytes of a box row (= swizzle span)
+  static constexpr int CPR = VROW / 16;               // 16-byte chunks per box row
+  static constexpr int CB = D_H / VW;                 // boxes per group
+  static constexpr int BOX = TT * VROW;               // bytes of one [TT x VW] bf16 box
   static constexpr int XB = NG * CB * BOX;            // scores operand (V or K)
   static constexpr int VB = GQA ? XB : 0;             // separate value tile (GQA)
   static constexpr int KRB = DRP ? TT * DRP * 2 : 0;  // positional key tile
@@ -116,7 +121,7 @@ struct MmaCfg {
   static_assert(STAGES % W == 0, "each stage must belong to one warp of a group");
   static_assert(W == 1 || P == 1, "round robin over tiles or rows split, not both");
   static_assert(MT % P == 0, "row parts must divide the tile's 16-row blocks");
-  static_assert(D_H % 64 == 0, "d_h");
+  static_assert(D_H == 32 || D_H % 64 == 0, "d_h");
   static_assert(DRP == 0 || DRP == 16 || DRP == 32, "padded d_r");
 
   static size_t smem_bytes(int B) {
@@ -212,13 +217,13 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
     for (int g = 0; g < C::NG; ++g)
 #pragma unroll
       for (int c = 0; c < C::CB; ++c)
-        tma_load_2d_hint(st + (g * C::CB + c) * C::BOX, &tm_x, g * C::D_H + c * 64, y, fb, pol);
+        tma_load_2d_hint(st + (g * C::CB + c) * C::BOX, &tm_x, g * C::D_H + c * C::VW, y, fb, pol);
     if constexpr (C::GQA) {
 #pragma unroll
       for (int g = 0; g < C::NG; ++g)
 #pragma unroll
         for (int c = 0; c < C::CB; ++c)
-          tma_load_2d_hint(st + C::XB + (g * C::CB + c) * C::BOX, &tm_v, g * C::D_H + c * 64, y, fb,
+          tma_load_2d_hint(st + C::XB + (g * C::CB + c) * C::BOX, &tm_v, g * C::D_H + c * C::VW, y, fb,
                            pol);
     }
     if constexpr (C::DRP > 0) tma_load_2d_hint(st + C::XB, &tm_kr, 0, y, fb, pol);
@@ -474,9 +479,9 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
         // rows past the sequence may hold anything (even NaN): zero this warp's
         // rows so that p = 0 really contributes nothing to P.V
         const int r0 = max(nvalid, r_lo), nz = r_hi - r0;
-        for (int e = lane; e < nz * 8 * C::CB; e += 32) {
-          const int c = e / (nz * 8), rr = r0 + (e >> 3) % nz, ch = e & 7;
-          *reinterpret_cast<uint4*>(vg + c * C::BOX + rr * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+        for (int e = lane; e < nz * C::CPR * C::CB; e += 32) {
+          const int c = e / (nz * C::CPR), rr = r0 + (e / C::CPR) % nz, ch = e % C::CPR;
+          *reinterpret_cast<uint4*>(vg + c * C::BOX + rr * C::VROW + ch * 16) = make_uint4(0, 0, 0, 0);
         }
         __syncwarp();
       }
@@ -497,7 +502,14 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
 #pragma unroll
         for (int ks = 0; ks < C::KS; ++ks) {
           uint32_t a0, a1, a2, a3;
-          ldsm_x4(xg_u + (ks >> 2) * C::BOX + arow * 128 + ((((ks & 3) * 2 + a_kc) ^ r8) << 4), a0,
+          // k-step ks covers columns [16 ks, 16 ks + 16): box ks / (CPR/2), chunk pair
+          // ks % (CPR/2); the swizzle XORs the chunk with row bits (rows of 128 bytes:
+          // row & 7, which is r8 here; of 64 bytes: (row >> 1) & 3)
+          const uint32_t xoff = C::VROW == 128
+              ? (ks >> 2) * C::BOX + arow * 128 + ((((ks & 3) * 2 + a_kc) ^ r8) << 4)
+              : (ks / (C::CPR / 2)) * C::BOX +
+                    swz<C::VROW>(arow * C::VROW + ((ks % (C::CPR / 2)) * 2 + a_kc) * 16);
+          ldsm_x4(xg_u + xoff, a0,
                   a1, a2, a3);
 #pragma unroll
           for (int nt = 0; nt < C::NT; ++nt)
@@ -531,8 +543,12 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       for (int mm = 0; mm < C::MW; ++mm)
 #pragma unroll
         for (int md = 0; md < C::KS; ++md)
-          ldsm_x4_t(vg_u + (md >> 2) * C::BOX + (v_tok + r_lo + mm * 16) * 128 +
-                        ((((md & 3) * 2 + v_dc) ^ r8) << 4),
+          ldsm_x4_t(vg_u + (C::VROW == 128
+                                ? (md >> 2) * C::BOX + (v_tok + r_lo + mm * 16) * 128 +
+                                      ((((md & 3) * 2 + v_dc) ^ r8) << 4)
+                                : (md / (C::CPR / 2)) * C::BOX +
+                                      swz<C::VROW>((v_tok + r_lo + mm * 16) * C::VROW +
+                                                   ((md % (C::CPR / 2)) * 2 + v_dc) * 16)),
                     vf[mm][md][0], vf[mm][md][1], vf[mm][md][2], vf[mm][md][3]);
 
       // ---- online softmax (fp32, base 2); this thread owns heads hcol, hcol+1
