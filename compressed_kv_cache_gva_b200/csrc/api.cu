@@ -143,6 +143,43 @@ gva_status_t plan_decode(const gva_shape_t& sh, bool gqa, long long max_total, P
   return GVA_OK;
 }
 
+// Every check of a decode call (sh already carries the nq * H heads), before
+// anything is launched; fills the plan.
+gva_status_t decode_check(const gva_shape_t& sh, bool gqa, const void* q, const void* X,
+                          const void* Vv, const void* KR, const int32_t* seq_offset,
+                          const int32_t* seq_len, int64_t max_total_tokens, int64_t num_slots,
+                          const void* out, const float* lse, const void* workspace,
+                          size_t ws_bytes, int nq, bool raw_q, Plan* pp) {
+  gva_status_t s;
+  Plan& p = *pp;
+  if (!q || !X || !Vv || !seq_offset || !seq_len || !out || !workspace)
+    return fail(GVA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!gqa && sh.d_r > 0 && !KR) return fail(GVA_ERR_INVALID_ARG, "kr_cache is NULL with d_r > 0");
+  if (!aligned16(q) || !aligned16(X) || !aligned16(Vv) || (KR && !aligned16(KR)) || !aligned16(out) ||
+      !aligned16(workspace) || !aligned16(seq_offset) || !aligned16(seq_len) || (lse && !aligned16(lse)))
+    return fail(GVA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (num_slots < 1 || num_slots >= (1ll << 31))
+    return fail(GVA_ERR_INVALID_ARG, "num_slots=%lld outside [1, 2^31)", (long long)num_slots);
+  if (max_total_tokens < 0 || max_total_tokens >= (1ll << 31))
+    return fail(GVA_ERR_INVALID_ARG, "max_total_tokens=%lld outside [0, 2^31)", (long long)max_total_tokens);
+  const int e = elt(sh.cache_dtype);
+  if ((sh.G * sh.d_h * e) % 16 || (!gqa && (sh.d_r * e) % 16))
+    return fail(GVA_ERR_INVALID_ARG, "cache rows must be multiples of 16 bytes (G*d_h*elt=%d, d_r*elt=%d)",
+                sh.G * sh.d_h * e, gqa ? 0 : sh.d_r * e);
+  if ((s = plan_decode(sh, gqa, max_total_tokens, &p, !gqa && !raw_q && nq == 1)) != GVA_OK)
+    return s;
+  if (nq > 1 && !p.mma)
+    return fail(GVA_ERR_UNSUPPORTED, "several query tokens need the tensor-core kernel "
+                "(bf16 cache, (H/G)*n_query <= 8, d_h in {32, 64, 128})");
+  if (ws_bytes < p.ws.total)
+    return fail(GVA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, p.ws.total);
+
+  if (!p.mma && !gva::simt_supported(sh, gqa))
+    return fail(GVA_ERR_UNSUPPORTED, "no decode kernel for H=%d G=%d d_h=%d d_r=%d", sh.H, sh.G,
+                sh.d_h, sh.d_r);
+  return GVA_OK;
+}
+
 gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, const void* X,
                            const void* Vv, const void* KR, const int32_t* seq_offset,
                            const int32_t* seq_len, int64_t max_total_tokens, int64_t num_slots,
@@ -159,28 +196,10 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
   shv.H = shp->H * nq;
   const gva_shape_t& sh = shv;
   if (sh.B == 0) return GVA_OK;
-  if (!q || !X || !Vv || !seq_offset || !seq_len || !out || !workspace)
-    return fail(GVA_ERR_INVALID_ARG, "a required pointer is NULL");
-  if (!gqa && sh.d_r > 0 && !KR) return fail(GVA_ERR_INVALID_ARG, "kr_cache is NULL with d_r > 0");
-  if (!aligned16(q) || !aligned16(X) || !aligned16(Vv) || (KR && !aligned16(KR)) || !aligned16(out) ||
-      !aligned16(workspace) || !aligned16(seq_offset) || !aligned16(seq_len) || (lse && !aligned16(lse)))
-    return fail(GVA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
-  if (num_slots < 1 || num_slots >= (1ll << 31))
-    return fail(GVA_ERR_INVALID_ARG, "num_slots=%lld outside [1, 2^31)", (long long)num_slots);
-  if (max_total_tokens < 0 || max_total_tokens >= (1ll << 31))
-    return fail(GVA_ERR_INVALID_ARG, "max_total_tokens=%lld outside [0, 2^31)", (long long)max_total_tokens);
-  const int e = elt(sh.cache_dtype);
-  if ((sh.G * sh.d_h * e) % 16 || (!gqa && (sh.d_r * e) % 16))
-    return fail(GVA_ERR_INVALID_ARG, "cache rows must be multiples of 16 bytes (G*d_h*elt=%d, d_r*elt=%d)",
-                sh.G * sh.d_h * e, gqa ? 0 : sh.d_r * e);
   Plan p;
-  if ((s = plan_decode(sh, gqa, max_total_tokens, &p, !gqa && !raw_q && nq == 1)) != GVA_OK)
+  if ((s = decode_check(sh, gqa, q, X, Vv, KR, seq_offset, seq_len, max_total_tokens, num_slots,
+                        out, lse, workspace, ws_bytes, nq, raw_q, &p)) != GVA_OK)
     return s;
-  if (nq > 1 && !p.mma)
-    return fail(GVA_ERR_UNSUPPORTED, "several query tokens need the tensor-core kernel "
-                "(bf16 cache, (H/G)*n_query <= 8, d_h in {64, 128})");
-  if (ws_bytes < p.ws.total)
-    return fail(GVA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, p.ws.total);
 
   gva::DecodeArgs a{};
   a.B = sh.B;
@@ -262,9 +281,6 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
     err = gva::launch_decode_mma(sh, gqa, a, tx, tv, tk, st);
   } else {
     a.tile = gva::simt_tile();
-    if (!gva::simt_supported(sh, gqa))
-      return fail(GVA_ERR_UNSUPPORTED, "no decode kernel for H=%d G=%d d_h=%d d_r=%d", sh.H, sh.G,
-                  sh.d_h, sh.d_r);
     if ((err = clear()) != cudaSuccess) return cuda_fail(err, "clearing the status word");
     err = gva::launch_decode_simt(sh, gqa, a, st);
     if (err == cudaErrorNotSupported)
@@ -424,12 +440,12 @@ gva_status_t gva_decode_step(const gva_shape_t* shape, const void* q, const void
   if (s != GVA_OK) return s;
   if (shape->B == 0 && n_new == 0) return GVA_OK;
   // Validate the decode first (it has the strictest requirements), without launching.
-  if (!q_abs || !V_cache || !seq_offset || !seq_len || !out || !workspace)
-    return fail(GVA_ERR_INVALID_ARG, "a required pointer is NULL");
   Plan p;
-  if ((s = plan_decode(*shape, false, max_total_tokens, &p, true)) != GVA_OK) return s;
-  if (ws_bytes < p.ws.total)
-    return fail(GVA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, p.ws.total);
+  if (shape->B > 0 &&
+      (s = decode_check(*shape, false, q_abs, V_cache, V_cache, kr_cache, seq_offset, seq_len,
+                        max_total_tokens, num_slots, out, lse, workspace, ws_bytes, 1, false, &p)) !=
+          GVA_OK)
+    return s;
   // 1. new tokens into the cache and absorbed queries (one kernel), 2. decode.
   // The first kernel lets the split kernel launch immediately and waits on the
   // preceding kernel before its first store; the split kernel streams every cache
@@ -614,13 +630,16 @@ gva_status_t gqa_decode_step(const gva_shape_t* shape, const void* q, const int3
   if (n_new > 0 &&
       (s = gqa_append_check(*shape, k_new, v_new, slot, pos, num_slots, K_cache, V_cache)) != GVA_OK)
     return s;
-  // the decode reads the rotated float32 query
+  // the decode reads the rotated float32 query; every check of it happens here,
+  // before the first launch
   gva_shape_t shd = *shape;
   shd.q_dtype = GVA_F32;
   Plan p;
-  if ((s = plan_decode(shd, true, max_total_tokens, &p, false)) != GVA_OK) return s;
-  if (ws_bytes < p.ws.total)
-    return fail(GVA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, p.ws.total);
+  if (shape->B > 0 &&
+      (s = decode_check(shd, true, q_rot, K_cache, V_cache, nullptr, seq_offset, seq_len,
+                        max_total_tokens, num_slots, out, lse, workspace, ws_bytes, 1, false, &p)) !=
+          GVA_OK)
+    return s;
   cudaError_t e = gva::launch_gqa_prep(*shape, q, q_pos, q_rot, n_new, k_new, v_new, slot, pos,
                                        num_slots, K_cache, V_cache, err_flag,
                                        static_cast<cudaStream_t>(stream));

@@ -156,6 +156,26 @@ def test_gqa_append_and_step_validate_on_the_host(L):
     assert st == 1 and b"NULL" in L.gva_last_error()
 
 
+def test_steps_check_the_decode_before_launching(L):
+    """gva_decode_step and gqa_decode_step run every check of their decode (pointers,
+    alignment, sizes) before their first kernel: a misaligned output or a bad cache
+    size is an INVALID_ARG status, not a launch followed by an error."""
+    sh = _shape()
+    st = L.gva_decode_step(ctypes.byref(sh), FAKE, FAKE, FAKE, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                           100, FAKE, FAKE, 100, FAKE, FAKE + 4, None, None, FAKE, 1 << 20, None)
+    assert st == 1 and b"aligned" in L.gva_last_error()
+    st = L.gva_decode_step(ctypes.byref(sh), FAKE, FAKE, FAKE, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                           0, FAKE, FAKE, 100, FAKE, FAKE, None, None, FAKE, 1 << 20, None)
+    assert st == 1 and b"num_slots" in L.gva_last_error()
+    shg = _shape(d_h=64, d_n=64, d_r=0)
+    st = L.gqa_decode_step(ctypes.byref(shg), FAKE, FAKE, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 100,
+                           FAKE, FAKE, 100, FAKE, FAKE + 8, None, None, FAKE, 1 << 20, None)
+    assert st == 1 and b"aligned" in L.gva_last_error()
+    st = L.gqa_decode_step(ctypes.byref(shg), FAKE, FAKE, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 100,
+                           FAKE, FAKE, 1 << 31, FAKE, FAKE, None, None, FAKE, 1 << 20, None)
+    assert st == 1 and b"max_total_tokens" in L.gva_last_error()
+
+
 def test_missing_library_fails_loudly(tmp_path):
     """No fallback: without the compiled library the binding raises on first use."""
     import subprocess
