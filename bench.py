@@ -603,21 +603,11 @@ def run_ours(args, rank, world, local):
     ms_e2e_serial, _, _ = timer.time_fn(e2e_step, K, R)
     ms_e2e = ms_e2e_serial
     e2e_mode = "serial: copy in, step, copy out, one after the other on one stream"
-    ms_pipe = ms_zero = None
     if not split_seq:
-        ms_pipe = time_e2e_pipelined(st, parts, h_stage, nb, view, K, dev, timer)
-        ms_zero = time_e2e_zero_copy(st, K, timer)
-        if ms_zero <= ms_pipe:
-            ms_e2e = ms_zero
-            e2e_mode = ("zero-copy: every step's first kernel reads the step's inputs from "
-                        "page-locked host memory over the bus and the combine writes its output "
-                        "into page-locked host memory; no copy nodes, so the step keeps its "
-                        "programmatic-launch chain")
-        else:
-            ms_e2e = ms_pipe
-            e2e_mode = ("pipelined: every step copies its inputs host->device and its output "
-                        "device->host on two copy streams, through two staging and output "
-                        "buffers, so the copies of one step overlap the compute of its neighbours")
+        ms_e2e = time_e2e_pipelined(st, parts, h_stage, nb, view, K, dev, timer)
+        e2e_mode = ("pipelined: every step copies its inputs host->device and its output "
+                    "device->host on two copy streams, through two staging and output buffers, "
+                    "so the copies of one step overlap the compute of its neighbours")
 
     workloads = {}
     extra = [] if (args.workloads in ("", "none") or split_seq or world > 1) else \
@@ -667,9 +657,7 @@ def run_ours(args, rank, world, local):
                 "ms_per_step": round(ms_e2e, 6), "mode": e2e_mode,
                 "serial": {"value": round(job_value(st.step_cache_bytes, 1, job_ranks,
                                                     ms_e2e_serial), 2),
-                           "ms_per_step": round(ms_e2e_serial, 6)},
-                "pipelined_copies_ms_per_step": None if ms_pipe is None else round(ms_pipe, 6),
-                "zero_copy_ms_per_step": None if ms_zero is None else round(ms_zero, 6)},
+                           "ms_per_step": round(ms_e2e_serial, 6)}},
         "multi_token": multi,
         "prefill": prefill,
         "workloads": workloads,
@@ -748,46 +736,6 @@ def time_e2e_pipelined(st, parts, h_stage, nb, view, K, dev, timer, nbuf=None):
     for k in range(NBUF):
         assert torch.equal(o_host[k], o_chk.cpu()), "pipelined end-to-end output differs"
     return ms / K
-
-
-def time_e2e_zero_copy(st, K, timer):
-    """End-to-end steps on page-locked host buffers that the kernels access directly,
-    ms per step.  Every step's inputs (query, new value, new positional key, slot,
-    position) are read by the step's first kernel from pinned host memory over the
-    bus, and the combine writes the step's output into pinned host memory: the same
-    bytes cross the bus every step as with explicit copies, but the graph has no
-    copy nodes, so the step's kernels keep their programmatic-dependent-launch
-    chain.  (With unified addressing, memory from cudaHostAlloc -- torch's pinned
-    memory -- is device-accessible through the same pointer.)  The C ABI is called
-    directly with those host pointers; the output that reached the host is checked
-    against a plain step's output."""
-    import ctypes
-    host = [t.contiguous().pin_memory() for t in [st.di.q] + st.app_host]
-    B, H, d_h = st.B, st.wl.H, st.wl.d_h
-    h_out = torch.empty(B, H, d_h, dtype=torch.float32).pin_memory()
-    L = gva.lib()
-    q, v_new, kpe_new, slot, pos = (t.data_ptr() for t in host)
-    n_new = host[3].numel()
-    ws_bytes = st.ws.numel()
-
-    def step(c):
-        rc = L.gva_decode_step(ctypes.byref(st.sh), q, st.M.data_ptr(), st.qpos.data_ptr(), n_new,
-                               v_new, kpe_new, slot, pos, st.Vs[c].data_ptr(),
-                               st.KRs[c].data_ptr(), st.Vs[c].shape[0], st.soff.data_ptr(),
-                               st.slen.data_ptr(), st.max_total, st.q_abs.data_ptr(),
-                               h_out.data_ptr(), None, None, st.ws.data_ptr(), ws_bytes,
-                               torch.cuda.current_stream().cuda_stream)
-        if rc != 0:
-            raise gva.GVAError(rc, L.gva_last_error().decode())
-
-    for c in range(st.R):
-        step(c)
-    ms, _, _ = timer.time_fn(step, K, st.R)
-    o_chk = torch.empty(B, H, d_h, dtype=torch.float32, device=st.dev)
-    st.step(0, o=o_chk)
-    torch.cuda.synchronize()
-    assert torch.equal(h_out, o_chk.cpu()), "zero-copy end-to-end output differs"
-    return ms
 
 
 def time_multi_token(st, Q, timer, K, dev, ms_dec):

@@ -251,12 +251,8 @@ gva_status_t gqa_decode_step(const gva_shape_t* shape, const void* q, const int3
  * [B, H, d_h + d_r] float32 buffer for the absorbed queries, err_flag may be NULL.
  * Because the append finishes before the decode is launched, the decode starts
  * streaming the cache while the absorb kernel still runs.  Validation of all three
- * parts happens before the first launch.
- * The per-step inputs q, v_new, kpe_new, slot and pos, and the outputs out and
- * lse, may also be page-locked host memory (cudaHostAlloc / cudaMallocHost) on a
- * system with unified addressing: the kernels then read and write them over the
- * bus directly, with no copy.  M, q_pos, the caches, q_abs, seq_offset, seq_len and
- * the workspace must be device memory.
+ * parts happens before the first launch, except for errors only the append or
+ * absorb checks catch, in which case the earlier parts may have been enqueued.
  */
 gva_status_t gva_decode_step(const gva_shape_t* shape, const void* q, const void* M,
                              const int32_t* q_pos, int32_t n_new, const void* v_new,
