@@ -29,6 +29,16 @@
  *     launched with programmatic stream serialization right after a call here
  *     must execute griddepcontrol.wait (cudaGridDependencySynchronize) before it
  *     reads that call's outputs; normally launched kernels need nothing.
+ *   - In the other direction, the first kernel of a call reads the call's inputs
+ *     (queries, key maps, new tokens, slots, positions, lengths, offsets, and in a
+ *     fused step the cache rows other than its new slots) before it waits for the
+ *     work before it on the stream, so that the reads overlap that work's tail.
+ *     A dependent may start once every thread block of the preceding kernel has
+ *     exited or triggered its dependents.  Inputs from copies, from calls of this
+ *     library, and from kernels that do not trigger dependents early and make their
+ *     stores visible before their blocks exit (a __threadfence() at the end of
+ *     the producer guarantees it) are complete by then.  A producer that triggers
+ *     early must do so only after those stores are visible.
  *   - Host-side validation happens before anything is launched; a non-OK status
  *     means nothing was enqueued.  gva_last_error() returns a one-line reason for
  *     the last non-OK status of the calling thread.  GVA_ERR_CUDA reports a launch
