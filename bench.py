@@ -239,14 +239,16 @@ class GraphTimer:
     def timed(self, gs):
         """Median device ms of one pass over `gs` (max over ranks), the number of
         passes and the host window."""
+        st = torch.cuda.current_stream()
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
-        c0 = time.perf_counter()
+        c0.record(st)
         for _ in range(3):                         # calibration passes (untimed)
             self.replay(gs)
+        c1.record(st)
         torch.cuda.synchronize()
-        n = passes_for((time.perf_counter() - c0) / 3)
+        n = passes_for(c0.elapsed_time(c1) / 3 * 1e-3)
         n = int(reduce_max(n, device=self.dev))    # the same count on every rank
-        st = torch.cuda.current_stream()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
         self.barrier()
         torch.cuda.synchronize()

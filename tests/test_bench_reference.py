@@ -43,3 +43,18 @@ def test_reference_other_ranks_silent():
     r = run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def test_timed_region_length():
+    """The K-step pass is replayed until at least 0.2 s and 20 passes have run:
+    the driver's short runs (K = 20, a ~0.2 ms pass) replay it ~1000 times."""
+    import importlib
+    import sys
+    sys.path.insert(0, ROOT)
+    bench = importlib.import_module("bench")
+    assert bench.passes_for(0.2e-3) == 1000
+    assert bench.passes_for(0.05) == 20            # long passes: the 20-pass floor
+    assert bench.passes_for(2.0) == 20
+    assert bench.passes_for(0.0) == bench.MAX_PASSES
+    args = bench.parse([])
+    assert args.steps >= 20 and args.warmup >= 3
