@@ -242,12 +242,14 @@ class GraphTimer:
         st = torch.cuda.current_stream()
         c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
+        self.replay(gs)                            # the first replays run slower
         c0.record(st)
-        for _ in range(3):                         # calibration passes (untimed)
+        for _ in range(8):                         # calibration passes (untimed)
             self.replay(gs)
         c1.record(st)
         torch.cuda.synchronize()
-        n = passes_for(c0.elapsed_time(c1) / 3 * 1e-3)
+        # 25% margin: the timed passes may run faster than the calibration ones
+        n = passes_for(c0.elapsed_time(c1) / 8 * 1e-3, min_s=1.25 * MIN_TIMED_S)
         n = int(reduce_max(n, device=self.dev))    # the same count on every rank
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
         self.barrier()
