@@ -184,7 +184,7 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
                            const void* Vv, const void* KR, const int32_t* seq_offset,
                            const int32_t* seq_len, int64_t max_total_tokens, int64_t num_slots,
                            void* out, float* lse, void* workspace, size_t ws_bytes, void* stream,
-                           bool prefetch = false, const int32_t* new_slots = nullptr,
+                           const int32_t* new_slots = nullptr,
                            int n_new = 0, int nq = 1, bool raw_q = false,
                            bool clear_status = false) {
   gva_status_t s = check_shape(shp, gqa);
@@ -226,7 +226,12 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
   a.part_ml = reinterpret_cast<float2*>(ws + p.ws.ml_off);
   a.part_o = reinterpret_cast<float*>(ws + p.ws.o_off);
   a.grid = p.grid;
-  a.prefetch = prefetch ? 1 : 0;
+  // Every decode requests its first cache tiles before its PDL wait: the cache
+  // rows are final by then (a fused step's own new slots excepted, listed in
+  // new_slots), since the kernels of this library that write cache rows let
+  // their successor launch only at their exit, or, in a fused step, only ahead
+  // of a split kernel that avoids those rows.
+  a.prefetch = 1;
   a.new_slots = new_slots;
   a.n_new = new_slots ? n_new : 0;
 #ifdef GVA_TRACE
@@ -310,7 +315,7 @@ gva_status_t decode_attention_clearing_status(const gva_shape_t* shape, const fl
                                               void* out, float* lse, void* workspace,
                                               size_t ws_bytes, void* stream) {
   return decode_common(shape, false, q_abs, V_cache, V_cache, kr_cache, seq_offset, seq_len,
-                       max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream, false,
+                       max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream,
                        nullptr, 0, 1, false, /*clear_status=*/true);
 }
 }  // namespace gva
@@ -466,8 +471,8 @@ gva_status_t gva_decode_step(const gva_shape_t* shape, const void* q, const void
   }
   if (shape->B == 0) return GVA_OK;
   return decode_common(shape, false, q_abs, V_cache, V_cache, kr_cache, seq_offset, seq_len,
-                       max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream,
-                       /*prefetch=*/true, slot, n_new);
+                       max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream, slot,
+                       n_new);
 }
 
 size_t gva_decode_workspace_size_multi(const gva_shape_t* shape, int32_t n_query,
@@ -537,7 +542,7 @@ gva_status_t gva_decode_attention_multi(const gva_shape_t* shape, int32_t n_quer
                           num_slots, out, lse, workspace, ws_bytes, stream);
   }
   return decode_common(shape, false, q_abs, V_cache, V_cache, kr_cache, seq_offset, seq_len,
-                       max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream, false,
+                       max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream,
                        nullptr, 0, n_query);
 }
 
@@ -552,7 +557,7 @@ gva_status_t gva_shared_kv_decode_attention(const gva_shape_t* shape, const void
                 shape->d_r, shape->d_n);
   // keys are the values (M_h = I): the raw query meets the value tile directly
   return decode_common(shape, false, q, V_cache, V_cache, nullptr, seq_offset, seq_len,
-                       max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream, false,
+                       max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream,
                        nullptr, 0, 1, /*raw_q=*/true);
 }
 
@@ -646,8 +651,8 @@ gva_status_t gqa_decode_step(const gva_shape_t* shape, const void* q, const int3
   if (e != cudaSuccess) return cuda_fail(e, "GQA query rotation + append launch");
   if (shape->B == 0) return GVA_OK;
   return decode_common(&shd, true, q_rot, K_cache, V_cache, nullptr, seq_offset, seq_len,
-                       max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream,
-                       /*prefetch=*/true, slot, n_new);
+                       max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream, slot,
+                       n_new);
 }
 
 gva_status_t gqa_decode_attention(const gva_shape_t* shape, const void* q, const void* K_cache,

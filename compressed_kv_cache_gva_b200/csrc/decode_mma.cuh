@@ -228,10 +228,12 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
     }
     if constexpr (C::DRP > 0) tma_load_2d_hint(st + C::XB, &tm_kr, 0, y, fb, pol);
   };
-  // Fused step only: every cache row except the ones this step appends is final
-  // before this kernel launches, so the first stages are requested before the
-  // PDL wait, up to the first tile of this CTA that uses an appended row.  All
-  // threads map the appended slots onto this CTA's tile ordinals in parallel.
+  // Every cache row is final before this kernel launches (the library's kernels
+  // that write cache rows let their successor launch only at their exit), except
+  // the rows a fused step's own first kernel appends: the first stages are
+  // requested before the PDL wait, up to the first tile of this CTA that uses an
+  // appended row.  All threads map the appended slots onto this CTA's tile
+  // ordinals in parallel.
   // (Rows a tile reads past its piece's end are never used, so only rows inside
   // the pieces count.)
   __shared__ int first_dirty;

@@ -276,8 +276,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       for (int g = 0; g < C::G; ++g) tma_load_2d_hint(st + C::VB + g * C::KR1, &tm_kr, 0, y, fb, pol);
     }
   };
-  // Fused step only: tiles without a row this step appends are final before this
-  // kernel launches and are requested before the PDL wait.
+  // Tiles without a row a fused step appends are final before this kernel
+  // launches and are requested before the PDL wait.
   __shared__ int first_dirty;
   if (a.prefetch) {
     if (threadIdx.x == 0) first_dirty = 0x7fffffff;

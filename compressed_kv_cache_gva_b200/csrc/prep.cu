@@ -196,7 +196,11 @@ __device__ __forceinline__ void append_block(long long bx, int N, int row_elems,
                 (double)pos[i], rt.inv_freq[p], y1[u], y2[u]);
   }
   pdl_wait();
-  if (!early_trigger) pdl_trigger();
+  // No trigger here: a decode streams cache rows before its own wait, so the
+  // kernel after a standalone append may launch only once the append's rows are
+  // stored (at its exit).  In a fused step the kernel triggers at entry and the
+  // split kernel leaves the appended rows alone until its wait.
+  (void)early_trigger;
   if (active && !ok) {
     if (lane == 0 && err_flag) atomicExch(err_flag, 1);
     return;
@@ -224,8 +228,8 @@ __global__ void append_cache_kernel(int N, int row_elems, int d_r, const T* __re
                                     T* __restrict__ V_cache, T* __restrict__ kr_cache,
                                     int* __restrict__ err_flag, const RopeTable rt,
                                     int early_trigger) {
-  // With early_trigger the successor may launch right away: it writes nothing
-  // this kernel reads, and it waits on this kernel before it depends on it.
+  // With early_trigger (never used by the standalone append) the successor could
+  // launch right away; without it the successor launches once this kernel exits.
   if (early_trigger) pdl_trigger();
   append_block<T>(blockIdx.x, N, row_elems, d_r, v_new, kpe_new, slot, pos, num_slots, V_cache,
                   kr_cache, err_flag, rt, early_trigger);
@@ -317,7 +321,11 @@ __device__ __forceinline__ void gqa_append_block(long long bx, int N, int G, int
     }
   }
   pdl_wait();
-  if (!early_trigger) pdl_trigger();
+  // No trigger here: a decode streams cache rows before its own wait, so the
+  // kernel after a standalone append may launch only once the append's rows are
+  // stored (at its exit).  In a fused step the kernel triggers at entry and the
+  // split kernel leaves the appended rows alone until its wait.
+  (void)early_trigger;
   if (active && !ok) {
     if (lane == 0 && err_flag) atomicExch(err_flag, 1);
     return;

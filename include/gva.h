@@ -30,9 +30,11 @@
  *     must execute griddepcontrol.wait (cudaGridDependencySynchronize) before it
  *     reads that call's outputs; normally launched kernels need nothing.
  *   - In the other direction, the first kernel of a call reads the call's inputs
- *     (queries, key maps, new tokens, slots, positions, lengths, offsets, and in a
- *     fused step the cache rows other than its new slots) before it waits for the
- *     work before it on the stream, so that the reads overlap that work's tail.
+ *     (queries, key maps, new tokens, slots, positions, lengths, offsets, and the
+ *     cache rows a decode attends, in a fused step those other than its new slots)
+ *     before it waits for the work before it on the stream, so that the reads
+ *     overlap that work's tail.  The append calls, which write cache rows, let the
+ *     next kernel launch only when they have completed.
  *     A dependent may start once every thread block of the preceding kernel has
  *     exited or triggered its dependents.  Inputs from copies, from calls of this
  *     library, and from kernels that do not trigger dependents early and make their

@@ -12,7 +12,8 @@ import torch
 import oracle
 from compressed_kv_cache_gva_b200 import gva
 from compressed_kv_cache_gva_b200.synth import (WORKLOADS, as_f64, make_append_inputs,
-                                                make_decode_inputs, make_gqa_inputs)
+                                                make_decode_inputs, make_gqa_append_inputs,
+                                                make_gqa_inputs)
 from gpu_helpers import (LOG2E, assert_close, dev, lse_close, oracle_gqa, oracle_gva, run_gqa,
                          run_gva, shape_of)
 
@@ -107,6 +108,90 @@ def test_append_then_decode_end_to_end():
     assert st == 0
     assert_close(out, ref, wl.dtype, "append+decode")
     lse_close(lse, ref_lse)
+
+
+@pytest.mark.parametrize("name", ["350m_b8_t4096", "dr24_b4_t32768"])
+def test_append_then_decode_without_sync(name):
+    """A decode requests its first cache tiles before its PDL wait; an append
+    launched just before it on the stream lets it launch only once the new rows
+    are stored.  Appended slots start out holding large garbage values, and each
+    decode follows its append with no synchronisation in between."""
+    wl = WORKLOADS[name]
+    lengths = np.array([40, 3, 100, 1])      # short: the new row sits in a CTA's first tiles
+    di = make_decode_inputs(wl, extra_slots=1, lengths=lengths)
+    offs = di.seq_offset.numpy()
+    slots = (offs + lengths).astype(np.int32)
+    V0, KR0 = di.V.clone(), di.k_rope.clone()
+    V0[torch.from_numpy(slots).long()] = 1000.0
+    KR0[torch.from_numpy(slots).long()] = 1000.0
+    ap = make_append_inputs(wl, slots, lengths.astype(np.int32))
+    seq_len = torch.from_numpy((lengths + 1).astype(np.int32))
+    q_pos = torch.from_numpy(lengths.astype(np.int32))
+    B, total = len(lengths), int(seq_len.sum())
+    sh = shape_of(di)
+    q_abs = torch.empty(B, wl.H, wl.d_h + wl.d_r, dtype=torch.float32, device="cuda")
+    gva.absorb_query(sh, dev(di.q), dev(di.M), dev(q_pos), q_abs)
+    soff, slen = dev(di.seq_offset), dev(seq_len)
+    v_new, kpe_new, slot, pos = dev(ap.v_new), dev(ap.kpe_new), dev(ap.slot), dev(ap.pos)
+    ws = gva.new_workspace(sh, total)
+    pairs = []
+    for _ in range(10):
+        V, KR = dev(V0), dev(KR0)
+        out = torch.empty(B, wl.H, wl.d_h, dtype=torch.float32, device="cuda")
+        lse = torch.empty(B, wl.H, dtype=torch.float32, device="cuda")
+        torch.cuda.synchronize()
+        gva.append_cache(sh, v_new, kpe_new, slot, pos, V, KR)
+        gva.decode_attention(sh, q_abs, V, KR, soff, slen, total, out, lse, ws)
+        pairs.append((out, lse))
+    torch.cuda.synchronize()
+    assert gva.workspace_status(ws) == 0
+    V_ref, K_ref, _ = oracle.append_cache(as_f64(V0), as_f64(KR0), as_f64(ap.v_new),
+                                          as_f64(ap.kpe_new), slots, lengths, wl.rope_base, wl.dtype)
+    ref, ref_lse = oracle.gva_decode(as_f64(di.q), as_f64(di.M), q_pos.numpy(), V_ref, K_ref, offs,
+                                     seq_len.numpy(), wl.d_n, wl.d_r, wl.rope_base)
+    for out, lse in pairs:
+        assert_close(out.cpu().numpy(), ref, wl.dtype, name)
+        lse_close(lse.cpu().numpy(), ref_lse, name)
+
+
+def test_gqa_append_then_decode_without_sync():
+    """The same for the GQA append and decode."""
+    wl = WORKLOADS["350m_b8_t4096"]
+    lengths = np.array([40, 3, 100, 1])
+    gi = make_gqa_inputs(wl, extra_slots=1, lengths=lengths)
+    offs = gi.seq_offset.numpy()
+    slots = (offs + lengths).astype(np.int32)
+    K0, V0 = gi.K.clone(), gi.V.clone()
+    K0[torch.from_numpy(slots).long()] = 1000.0
+    V0[torch.from_numpy(slots).long()] = 1000.0
+    ap = make_gqa_append_inputs(wl, slots, lengths.astype(np.int32))
+    seq_len = torch.from_numpy((lengths + 1).astype(np.int32))
+    B, total = len(lengths), int(seq_len.sum())
+    sh = gva.make_shape(B, wl.H, wl.G, wl.d_h, wl.d_h, 0, cache_dtype=wl.torch_dtype,
+                        rope_base=wl.rope_base)
+    q = dev(gi.q)
+    soff, slen = dev(gi.seq_offset), dev(seq_len)
+    ws = gva.new_workspace(sh, total)
+    outs = []
+    for _ in range(10):
+        K, V = dev(K0), dev(V0)
+        out = torch.empty(B, wl.H, wl.d_h, dtype=torch.float32, device="cuda")
+        torch.cuda.synchronize()
+        gva.gqa_append_cache(sh, dev(ap.k_new), dev(ap.v_new), dev(ap.slot), dev(ap.pos), K, V)
+        gva.gqa_decode_attention(sh, q, K, V, soff, slen, total, out, None, ws)
+        outs.append((out, K))
+    torch.cuda.synchronize()
+    assert gva.workspace_status(ws) == 0
+    K_ref, V_ref, _ = oracle.gqa_append_cache(as_f64(K0), as_f64(V0), as_f64(ap.k_new),
+                                              as_f64(ap.v_new), slots, lengths, wl.rope_base,
+                                              wl.dtype)
+    from compressed_kv_cache_gva_b200.synth import GQAInputs
+    ref, _ = oracle_gqa(GQAInputs(seq_len=seq_len, seq_offset=gi.seq_offset, q=gi.q,
+                                  K=torch.from_numpy(K_ref), V=torch.from_numpy(V_ref),
+                                  num_slots=gi.num_slots))
+    for out, K in outs:
+        assert np.array_equal(as_f64(K.cpu()), K_ref)
+        assert_close(out.cpu().numpy(), ref, wl.dtype, "gqa")
 
 
 # ------------------------------------------------------------------ decode
