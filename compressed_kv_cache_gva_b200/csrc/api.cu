@@ -186,7 +186,7 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
                            void* out, float* lse, void* workspace, size_t ws_bytes, void* stream,
                            const int32_t* new_slots = nullptr,
                            int n_new = 0, int nq = 1, bool raw_q = false,
-                           bool clear_status = false) {
+                           bool clear_status = false, bool step = false) {
   gva_status_t s = check_shape(shp, gqa);
   if (s != GVA_OK) return s;
   if (nq < 1 || nq > 64) return fail(GVA_ERR_INVALID_ARG, "n_query=%d outside [1,64]", nq);
@@ -232,6 +232,10 @@ gva_status_t decode_common(const gva_shape_t* shp, bool gqa, const void* q, cons
   // their successor launch only at their exit, or, in a fused step, only ahead
   // of a split kernel that avoids those rows.
   a.prefetch = 1;
+  // The queries of a plain decode are caller inputs, final before it launches
+  // (the library's absorb lets its successor launch only at its exit); in a fused
+  // step the first kernel writes them.
+  a.q_early = step ? 0 : 1;
   a.new_slots = new_slots;
   a.n_new = new_slots ? n_new : 0;
 #ifdef GVA_TRACE
@@ -472,7 +476,7 @@ gva_status_t gva_decode_step(const gva_shape_t* shape, const void* q, const void
   if (shape->B == 0) return GVA_OK;
   return decode_common(shape, false, q_abs, V_cache, V_cache, kr_cache, seq_offset, seq_len,
                        max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream, slot,
-                       n_new);
+                       n_new, 1, false, false, /*step=*/true);
 }
 
 size_t gva_decode_workspace_size_multi(const gva_shape_t* shape, int32_t n_query,
@@ -652,7 +656,7 @@ gva_status_t gqa_decode_step(const gva_shape_t* shape, const void* q, const int3
   if (shape->B == 0) return GVA_OK;
   return decode_common(&shd, true, q_rot, K_cache, V_cache, nullptr, seq_offset, seq_len,
                        max_total_tokens, num_slots, out, lse, workspace, ws_bytes, stream, slot,
-                       n_new);
+                       n_new, 1, false, false, /*step=*/true);
 }
 
 gva_status_t gqa_decode_attention(const gva_shape_t* shape, const void* q, const void* K_cache,

@@ -94,6 +94,7 @@ struct DecodeArgs {
   int nq;                    // query tokens per sequence (causal among them), >= 1
   int grid;                  // CTAs of the split kernel
   int tile;                  // span granularity in tokens
+  int q_early;               // read the queries before the PDL wait (no kernel of the call writes them)
   int prefetch;              // stream the cache before the PDL wait, except
   const int* new_slots;      //   tiles holding one of these n_new slots, written by the
   int n_new;                 //   append of the same step

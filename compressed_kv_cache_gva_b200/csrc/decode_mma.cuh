@@ -130,6 +130,87 @@ struct MmaCfg {
   }
 };
 
+// Query fragments of sequence b for consumer lane (gq, t) of group g (the B
+// operand of the score MMA, column n = gq): the absorbed fp32 query
+// (pre-scaled), or the raw query in its storage type, scaled here (GQA, and
+// GVA with shared keys and values: M = I, d_r = 0), split into bf16 hi / lo.
+// Padding columns (past the group's ncol real ones) get a zero query.
+template <class C>
+__device__ __forceinline__ void load_query(const DecodeArgs& a, const int b, const int g,
+                                           const int hpr, const int ncol, const int gq,
+                                           const int t, uint32_t (&qbo)[C::NT][C::KS][2],
+                                           uint32_t (&qro)[C::NT][C::RS > 0 ? C::RS : 1][2]) {
+  const int H = a.H, dq = C::D_H + a.d_r;
+#pragma unroll
+  for (int nt = 0; nt < C::NT; ++nt) {
+    const int hl = C::HPG == 8 ? gq : (gq & 3);     // column within the group
+    const bool lo = C::HPG == 8 ? (nt == 1) : (gq >= 4);
+    const int vq = hl / hpr, head = g * hpr + hl % hpr;
+    float v[C::KS][4];
+    float wv[C::RS > 0 ? C::RS : 1][4];
+    if (hl >= ncol) {   // padding column: zero query
+#pragma unroll
+      for (int ks = 0; ks < C::KS; ++ks)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[ks][e] = 0.f;
+#pragma unroll
+      for (int rs = 0; rs < (C::RS > 0 ? C::RS : 1); ++rs)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) wv[rs][e] = 0.f;
+    } else if (!C::GQA && a.q_raw == nullptr) {
+      const float* qrow = a.q_abs + (((size_t)b * a.nq + vq) * H + head) * dq;
+#pragma unroll
+      for (int ks = 0; ks < C::KS; ++ks) {
+        const int k0 = ks * 16 + 2 * t;
+        const float2 x01 = *reinterpret_cast<const float2*>(qrow + k0);
+        const float2 x89 = *reinterpret_cast<const float2*>(qrow + k0 + 8);
+        v[ks][0] = x01.x;
+        v[ks][1] = x01.y;
+        v[ks][2] = x89.x;
+        v[ks][3] = x89.y;
+      }
+#pragma unroll
+      for (int rs = 0; rs < C::RS; ++rs) {
+        const int k0 = rs * 16 + 2 * t;
+        wv[rs][0] = k0 < a.d_r ? qrow[C::D_H + k0] : 0.f;
+        wv[rs][1] = k0 + 1 < a.d_r ? qrow[C::D_H + k0 + 1] : 0.f;
+        wv[rs][2] = k0 + 8 < a.d_r ? qrow[C::D_H + k0 + 8] : 0.f;
+        wv[rs][3] = k0 + 9 < a.d_r ? qrow[C::D_H + k0 + 9] : 0.f;
+      }
+    } else {
+      const void* rawrow = reinterpret_cast<const char*>(a.q_raw) +
+          (((size_t)b * a.nq + vq) * H + head) * C::D_H * (a.q_bf16 ? 2 : 4);
+#pragma unroll
+      for (int ks = 0; ks < C::KS; ++ks) {
+        const int k0 = ks * 16 + 2 * t;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int kk = k0 + (e & 1) + (e >> 1) * 8;
+          const float x = a.q_bf16
+              ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(rawrow)[kk])
+              : reinterpret_cast<const float*>(rawrow)[kk];
+          v[ks][e] = x * a.q_scale;
+        }
+      }
+#pragma unroll
+      for (int rs = 0; rs < (C::RS > 0 ? C::RS : 1); ++rs)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) wv[rs][e] = 0.f;
+    }
+    auto part = [&](float x) { const float h = bf16_round(x); return lo ? x - h : h; };
+#pragma unroll
+    for (int ks = 0; ks < C::KS; ++ks) {
+      qbo[nt][ks][0] = pack_bf16(part(v[ks][0]), part(v[ks][1]));
+      qbo[nt][ks][1] = pack_bf16(part(v[ks][2]), part(v[ks][3]));
+    }
+#pragma unroll
+    for (int rs = 0; rs < C::RS; ++rs) {
+      qro[nt][rs][0] = pack_bf16(part(wv[rs][0]), part(wv[rs][1]));
+      qro[nt][rs][1] = pack_bf16(part(wv[rs][2]), part(wv[rs][3]));
+    }
+  }
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, C::MINB)
     decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_x,
@@ -265,6 +346,19 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       }
     }
   }
+  // query fragments (B operand of the score MMA), column n = gq, of sequence q_seq
+  uint32_t qb[C::NT][C::KS][2];
+  uint32_t qr[C::NT][C::RS > 0 ? C::RS : 1][2];
+  int q_seq = -1;
+  // A plain decode call's queries are its own inputs (no kernel of the call
+  // writes them): the consumers load their first sequence's query before the
+  // PDL wait, off the critical path.  In a fused step the first kernel writes
+  // them, so they wait.
+  if (a.q_early && warp < C::NCW && has_work && rng.reaches(b_first)) {
+    const int hpr0 = a.H / a.G;
+    load_query<C>(a, b_first, warp / C::GW, hpr0, hpr0 * a.nq, lane >> 2, lane & 3, qb, qr);
+    q_seq = b_first;
+  }
   pdl_wait();
   pdl_trigger();
   if (threadIdx.x == 0) trace_mark(a, 1);
@@ -363,85 +457,12 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
   bool ok = true;   // false once a bounded wait gave up: skip work, keep barrier order
 
   int k = 0;
-  // query fragments (B operand of the score MMA), column n = gq, of sequence q_seq
-  uint32_t qb[C::NT][C::KS][2];
-  uint32_t qr[C::NT][C::RS > 0 ? C::RS : 1][2];
-  int q_seq = -1;
   // One piece: tokens [j0, j1) of sequence b, tiles k, k+1, ... of the ring;
   // its partial state goes to `slot`.
   auto run_piece = [&](const int b, const int j0, const int j1, const size_t slot) {
     if (b != q_seq) {
-    q_seq = b;
-#pragma unroll
-    for (int nt = 0; nt < C::NT; ++nt) {
-      const int hl = C::HPG == 8 ? gq : (gq & 3);     // column within the group
-      const bool lo = C::HPG == 8 ? (nt == 1) : (gq >= 4);
-      const int vq = hl / hpr, head = g * hpr + hl % hpr;
-      float v[C::KS][4];
-      float wv[C::RS > 0 ? C::RS : 1][4];
-      // absorbed fp32 query (pre-scaled), or the raw query in its storage type,
-      // scaled here: GQA, and GVA with shared keys and values (M = I, d_r = 0)
-      if (hl >= ncol) {   // padding column: zero query
-#pragma unroll
-        for (int ks = 0; ks < C::KS; ++ks)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) v[ks][e] = 0.f;
-#pragma unroll
-        for (int rs = 0; rs < (C::RS > 0 ? C::RS : 1); ++rs)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) wv[rs][e] = 0.f;
-      } else if (!C::GQA && a.q_raw == nullptr) {
-        const float* qrow = a.q_abs + (((size_t)b * a.nq + vq) * H + head) * dq;
-#pragma unroll
-        for (int ks = 0; ks < C::KS; ++ks) {
-          const int k0 = ks * 16 + 2 * t;
-          const float2 x01 = *reinterpret_cast<const float2*>(qrow + k0);
-          const float2 x89 = *reinterpret_cast<const float2*>(qrow + k0 + 8);
-          v[ks][0] = x01.x;
-          v[ks][1] = x01.y;
-          v[ks][2] = x89.x;
-          v[ks][3] = x89.y;
-        }
-#pragma unroll
-        for (int rs = 0; rs < C::RS; ++rs) {
-          const int k0 = rs * 16 + 2 * t;
-          wv[rs][0] = k0 < a.d_r ? qrow[C::D_H + k0] : 0.f;
-          wv[rs][1] = k0 + 1 < a.d_r ? qrow[C::D_H + k0 + 1] : 0.f;
-          wv[rs][2] = k0 + 8 < a.d_r ? qrow[C::D_H + k0 + 8] : 0.f;
-          wv[rs][3] = k0 + 9 < a.d_r ? qrow[C::D_H + k0 + 9] : 0.f;
-        }
-      } else {
-        const void* rawrow = reinterpret_cast<const char*>(a.q_raw) +
-            (((size_t)b * a.nq + vq) * H + head) * C::D_H * (a.q_bf16 ? 2 : 4);
-#pragma unroll
-        for (int ks = 0; ks < C::KS; ++ks) {
-          const int k0 = ks * 16 + 2 * t;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int kk = k0 + (e & 1) + (e >> 1) * 8;
-            const float x = a.q_bf16
-                ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(rawrow)[kk])
-                : reinterpret_cast<const float*>(rawrow)[kk];
-            v[ks][e] = x * a.q_scale;
-          }
-        }
-#pragma unroll
-        for (int rs = 0; rs < (C::RS > 0 ? C::RS : 1); ++rs)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) wv[rs][e] = 0.f;
-      }
-      auto part = [&](float x) { const float h = bf16_round(x); return lo ? x - h : h; };
-#pragma unroll
-      for (int ks = 0; ks < C::KS; ++ks) {
-        qb[nt][ks][0] = pack_bf16(part(v[ks][0]), part(v[ks][1]));
-        qb[nt][ks][1] = pack_bf16(part(v[ks][2]), part(v[ks][3]));
-      }
-#pragma unroll
-      for (int rs = 0; rs < C::RS; ++rs) {
-        qr[nt][rs][0] = pack_bf16(part(wv[rs][0]), part(wv[rs][1]));
-        qr[nt][rs][1] = pack_bf16(part(wv[rs][2]), part(wv[rs][3]));
-      }
-    }
+      load_query<C>(a, b, g, hpr, ncol, gq, t, qb, qr);
+      q_seq = b;
     }
 
     // O^T fragments: d rows x 8 columns.  With 8 columns per group the hi and lo

@@ -120,7 +120,6 @@ __device__ __forceinline__ void absorb_block(int h, int by, int bz, int B, int H
       for (int k = 0; k < d_n; ++k) acc0 = fmaf(qv[k], to_f32(row[k]), acc0);
     }
     pdl_wait();
-    if (!early_trigger) pdl_trigger();
     if (row_ok) o[i] = (acc0 + acc1) * c;
   } else {
     const int half = d_r / 2;
@@ -135,7 +134,6 @@ __device__ __forceinline__ void absorb_block(int h, int by, int bz, int B, int H
                   y2[u]);
     }
     pdl_wait();
-    if (!early_trigger) pdl_trigger();
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int p = lane + 32 * u;
@@ -154,10 +152,13 @@ __global__ void __launch_bounds__(2 * kAbsorbQueries * 32)
                         float* __restrict__ q_abs, const RopeTable rt, int early_trigger) {
   extern __shared__ float sm[];
   // With early_trigger the successor may launch right away: it waits on this
-  // kernel before it reads q_abs.
+  // kernel before it reads q_abs.  A standalone absorb does not trigger: the
+  // next kernel launches once every block has exited, its stores made visible
+  // first, since a decode reads its query before its own wait.
   if (early_trigger) pdl_trigger();
   absorb_block<TQ>(blockIdx.x, blockIdx.y, blockIdx.z, B, H, d_h, d_n, d_r, c, q, M, q_pos, q_abs,
                    rt, sm, early_trigger);
+  if (!early_trigger) __threadfence();
 }
 
 // One warp per token: the value row is loaded (16-byte vectors) and the
@@ -229,10 +230,13 @@ __global__ void append_cache_kernel(int N, int row_elems, int d_r, const T* __re
                                     int* __restrict__ err_flag, const RopeTable rt,
                                     int early_trigger) {
   // With early_trigger (never used by the standalone append) the successor could
-  // launch right away; without it the successor launches once this kernel exits.
+  // launch right away; without it the successor launches once every block has
+  // exited, its stores made visible first (a decode streams cache rows before
+  // its own wait).
   if (early_trigger) pdl_trigger();
   append_block<T>(blockIdx.x, N, row_elems, d_r, v_new, kpe_new, slot, pos, num_slots, V_cache,
                   kr_cache, err_flag, rt, early_trigger);
+  if (!early_trigger) __threadfence();
 }
 
 // The first two kernels of the fused decode step in one launch: blocks
@@ -405,8 +409,11 @@ __global__ void __launch_bounds__(256)
                       const T* __restrict__ v_new, const int* __restrict__ slot,
                       const int* __restrict__ pos, long long num_slots, T* __restrict__ K_cache,
                       T* __restrict__ V_cache, int* __restrict__ err_flag, const RopeTable rt) {
+  // no trigger: the successor launches once every block has exited, its stores
+  // made visible first (a decode streams cache rows before its own wait)
   gqa_append_block<T>(blockIdx.x, N, G, d_h, k_new, v_new, slot, pos, num_slots, K_cache, V_cache,
                       err_flag, rt, 0);
+  __threadfence();
 }
 
 // The first kernel of the GQA decode step, the counterpart of prep_step_kernel:
