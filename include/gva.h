@@ -33,8 +33,9 @@
  *     (queries, key maps, new tokens, slots, positions, lengths, offsets, and the
  *     cache rows a decode attends, in a fused step those other than its new slots)
  *     before it waits for the work before it on the stream, so that the reads
- *     overlap that work's tail.  The append calls, which write cache rows, let the
- *     next kernel launch only when they have completed.
+ *     overlap that work's tail.  The append and absorb calls, whose outputs (cache
+ *     rows, absorbed queries) the next decode reads that early, let the next
+ *     kernel launch only when they have completed.
  *     A dependent may start once every thread block of the preceding kernel has
  *     exited or triggered its dependents.  Inputs from copies, from calls of this
  *     library, and from kernels that do not trigger dependents early and make their
