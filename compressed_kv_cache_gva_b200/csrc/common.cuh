@@ -116,15 +116,21 @@ __device__ __forceinline__ void trace_mark(const DecodeArgs& a, int slot) {
 #endif
 }
 
-// Per-tile timeline (same build flag): for the first 8 tiles of each CTA of the
-// split kernel, trace[65536 + (cta * 8 + k) * 4 + which] holds %globaltimer when
-// tile k was requested (which = 0), ready for group 0 (1) and released by it (2).
+// Per-tile timeline (same build flag): for the first 16 tiles of each of the
+// first 2048 CTAs of the split kernel, trace[65536 + (cta * 16 + k) * 4 + which]
+// holds %globaltimer when tile k was requested (which = 0), ready for group 0 (1)
+// and released by it (2); trace[200000 + cta] holds the CTA's SM.
 __device__ __forceinline__ void trace_tile(const DecodeArgs& a, int k, int which) {
 #ifdef GVA_TRACE
-  if (a.trace && k < 8) {
+  if (a.trace && k < 16 && blockIdx.x < 2048) {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    a.trace[65536 + (blockIdx.x * 8 + k) * 4 + which] = t;
+    a.trace[65536 + (blockIdx.x * 16 + k) * 4 + which] = t;
+    if (k == 0 && which == 0) {
+      unsigned sm;
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+      a.trace[200000 + blockIdx.x] = sm;
+    }
   }
 #else
   (void)a;

@@ -482,15 +482,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
     for (int t0 = j0; t0 < j1; t0 += C::TT, ++k) {
       if (k % C::W != w) continue;                 // another warp of the group takes it
       const int s = k % C::STAGES;
-#ifdef GVA_TRACE
-      const long long tw0 = clock64();
-#endif
       if (ok) ok = mbar_wait(smem_u32(full + s), (k / C::STAGES) & 1, a.status);
       if (!ok) continue;
-#ifdef GVA_TRACE
-      const long long tw1 = clock64();
-      if (warp == 0 && lane == 0 && a.trace) a.trace[blockIdx.x * 8 + 6] += (unsigned long long)(tw1 - tw0);
-#endif
       if (warp == 0 && lane == 0 && k == 0) trace_mark(a, 3);
       if (warp == 0 && lane == 0) trace_tile(a, k, 1);
       const int nvalid = min(C::TT, j1 - t0);
@@ -635,10 +628,6 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(empty + s));
       if (warp == 0 && lane == 0) trace_tile(a, k, 2);
-#ifdef GVA_TRACE
-      if (warp == 0 && lane == 0 && a.trace)
-        a.trace[blockIdx.x * 8 + 7] += (unsigned long long)(clock64() - tw1);
-#endif
     }
 
     // ---- piece epilogue
