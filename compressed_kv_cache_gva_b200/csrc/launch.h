@@ -56,7 +56,9 @@ cudaError_t launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, 
   return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
 }
 
-// early_trigger: let the next kernel launch at once (fused step only, see api.cu).
+// early_trigger: let the next kernel launch at once.  The library's own calls pass
+// false: the next kernel then launches once this one has exited with its stores
+// made visible, since a decode reads the queries and cache rows before its wait.
 cudaError_t launch_absorb(const gva_shape_t& sh, const void* q, const void* M, const int* q_pos,
                           float* q_abs, float c, cudaStream_t st, bool early_trigger = false);
 size_t absorb_smem_bytes(const gva_shape_t& sh);
