@@ -372,13 +372,11 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
     // depth in flight: one stage fewer for short ranges (tile k waits for tile
     // k - depth's release; consumers release in order, and that stage is not
     // refilled before tile k, so its barrier is still in that tile's phase).
-    // Only with one consumer warp per group: the stages armed before the PDL
-    // wait were armed unchecked, so the first tile armed here relies on the
-    // release of tile k - depth implying that of tile k - STAGES, the previous
-    // occupant of its stage; with W > 1 the warps of a group release alternate
-    // tiles in no fixed order and it does not (tile k could be armed on a
-    // barrier whose previous copy is still landing).  Those configurations wait
-    // for tile k - STAGES itself.  (A model of the protocol runs in the tests.)
+    // Only with one consumer warp per group: with W > 1 the warps of a group
+    // release alternate tiles in no fixed order, so the release of tile
+    // k - depth says nothing about tile k - STAGES, whose stage tile k reuses
+    // (its copy could still be landing when tile k's is armed on the same
+    // barrier); those configurations wait for tile k - STAGES itself.
     const int depth = (C::W == 1 && C::STAGES >= 4 && GVA_SHORT_RANGE_TILES > 0 &&
                        rng.T1 - rng.T0 <= GVA_SHORT_RANGE_TILES) ? C::STAGES - 1 : C::STAGES;
     for (; cur.b < a.B; ++k) {
