@@ -154,6 +154,71 @@ def test_append_then_decode_without_sync(name):
         lse_close(lse.cpu().numpy(), ref_lse, name)
 
 
+def test_absorb_then_decode_without_sync():
+    """A plain decode reads its absorbed queries before its PDL wait; the absorb
+    launched just before it lets it launch only once the queries are stored.
+    Every iteration absorbs a different query into the same buffer (which held
+    garbage first) and decodes at once, with no synchronisation."""
+    wl = WORKLOADS["350m_b8_t4096"]
+    di = small("350m_b8_t4096", lengths=[700, 33, 1500, 64])
+    sh = shape_of(di)
+    B, total = len(di.seq_len), di.total_tokens
+    V, KR = dev(di.V), dev(di.k_rope)
+    soff, slen, M, qpos = dev(di.seq_offset), dev(di.seq_len), dev(di.M), dev(di.q_pos)
+    q_abs = torch.full((B, wl.H, wl.d_h + wl.d_r), 1e4, dtype=torch.float32, device="cuda")
+    ws = gva.new_workspace(sh, total)
+    rng = np.random.default_rng(21)
+    qs, outs = [], []
+    for _ in range(6):
+        q = torch.from_numpy(rng.standard_normal(tuple(di.q.shape)).astype(np.float32)).to(di.q.dtype)
+        out = torch.empty(B, wl.H, wl.d_h, dtype=torch.float32, device="cuda")
+        gva.absorb_query(sh, dev(q), M, qpos, q_abs)
+        gva.decode_attention(sh, q_abs, V, KR, soff, slen, total, out, None, ws)
+        qs.append(q)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert gva.workspace_status(ws) == 0
+    for q, out in zip(qs, outs):
+        di.q = q
+        ref, _ = oracle_gva(di)
+        assert_close(out.cpu().numpy(), ref, wl.dtype, "absorb->decode")
+
+
+def test_decode_step_then_decode_without_sync():
+    """A fused step (its first kernel appends and absorbs, then the decode), then
+    a plain decode of the same batch on the step's absorbed queries and updated
+    cache, issued at once: the plain decode reads both before its own wait."""
+    wl = WORKLOADS["350m_b8_t4096"]
+    lengths = np.array([300, 65, 1, 1031])
+    di = make_decode_inputs(wl, extra_slots=1, lengths=lengths)
+    V0, K0 = as_f64(di.V), as_f64(di.k_rope)
+    offs = di.seq_offset.numpy()
+    slots = (offs + lengths).astype(np.int32)
+    ap = make_append_inputs(wl, slots, lengths.astype(np.int32))
+    seq_len = torch.from_numpy((lengths + 1).astype(np.int32))
+    q_pos = torch.from_numpy(lengths.astype(np.int32))
+    B, total = len(lengths), int(seq_len.sum())
+    sh = shape_of(di)
+    V, KR = dev(di.V), dev(di.k_rope)
+    q_abs = torch.empty(B, wl.H, wl.d_h + wl.d_r, dtype=torch.float32, device="cuda")
+    out1 = torch.empty(B, wl.H, wl.d_h, dtype=torch.float32, device="cuda")
+    out2 = torch.empty_like(out1)
+    ws1, ws2 = gva.new_workspace(sh, total), gva.new_workspace(sh, total)
+    soff, slen = dev(di.seq_offset), dev(seq_len)
+    gva.decode_step(sh, dev(di.q), dev(di.M), dev(q_pos), dev(ap.v_new), dev(ap.kpe_new),
+                    dev(ap.slot), dev(ap.pos), V, KR, soff, slen, total, q_abs, out1, None, None, ws1)
+    gva.decode_attention(sh, q_abs, V, KR, soff, slen, total, out2, None, ws2)
+    torch.cuda.synchronize()
+    assert gva.workspace_status(ws1) == 0 and gva.workspace_status(ws2) == 0
+    V_ref, K_ref, _ = oracle.append_cache(V0, K0, as_f64(ap.v_new), as_f64(ap.kpe_new), slots, lengths,
+                                          wl.rope_base, wl.dtype)
+    ref, _ = oracle.gva_decode(as_f64(di.q), as_f64(di.M), q_pos.numpy(), V_ref, K_ref, offs,
+                               seq_len.numpy(), wl.d_n, wl.d_r, wl.rope_base)
+    assert_close(out1.cpu().numpy(), ref, wl.dtype, "step")
+    assert_close(out2.cpu().numpy(), ref, wl.dtype, "decode after step")
+    assert torch.equal(out1, out2)
+
+
 def test_gqa_append_then_decode_without_sync():
     """The same for the GQA append and decode."""
     wl = WORKLOADS["350m_b8_t4096"]
